@@ -1,0 +1,160 @@
+"""Pins of the oracle's SIP sampler (inclusion probabilities and draws).
+
+Page: AB-Attention summary (news.hamidun.com), "AB-Attention's three
+techniques", SIP paragraph: inclusion probability proportional to score, the
+top blocks always taken, every block a nonzero chance.  Pins: the exact
+integer identity sum(pi) = n, an independent fp64 bisection of
+sum_j min(1, lambda q_j) = n, the published SplitMix64 outputs, and a
+frequency test of the draws.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from block_sparse_attention_selector_b200 import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def pis(s, n):
+    capped, r, R, _ = oracle.pi_solve(s, n)
+    q = oracle.quantised_scores(s)
+    return [1.0 if c else r * qj / R for c, qj in zip(capped, q)], capped, r, R, q
+
+
+@pytest.mark.parametrize("seed,nkb,n", [(0, 128, 13), (1, 500, 40), (2, 8190, 819), (3, 64, 63),
+                                        (4, 64, 1), (5, 1000, 400)])
+def test_pi_sums_to_budget_exactly_and_caps_are_the_fixed_point(seed, nkb, n):
+    s = synthetic.random_scores(1, nkb, seed)[0]
+    capped, r, R, rounds = oracle.pi_solve(s, n)
+    q = oracle.quantised_scores(s)
+    # exact: |C| + r * (sum of uncapped q) / R = |C| + r = n
+    assert int(capped.sum()) + r == n
+    assert R == sum(qj for qj, c in zip(q, capped) if not c)
+    for qj, c in zip(q, capped):
+        assert (r * qj >= R) == bool(c)  # fixed point: capped <=> r q_j >= R
+        if not c:
+            assert 0 < r * qj < R  # 0 < pi < 1
+    assert rounds >= 1
+
+
+def _bisection_pi(q, n):
+    """Independent characterisation: pi_j = min(1, lam q_j) with sum pi = n (fp64)."""
+    q = np.asarray(q, np.float64)
+    lo, hi = 0.0, n / q.min()
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if np.minimum(1.0, mid * q).sum() < n:
+            lo = mid
+        else:
+            hi = mid
+    return np.minimum(1.0, hi * q)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_pi_matches_bisection_brute_force(seed):
+    nkb = [16, 32, 64, 100, 128, 200][seed]
+    n = [3, 5, 13, 20, 50, 199][seed]
+    s = synthetic.random_scores(1, nkb, 100 + seed, concentration=2.0 + seed)[0]
+    p, capped, _, _, q = pis(s, n)
+    ref = _bisection_pi(q, n)
+    np.testing.assert_allclose(p, ref, rtol=1e-9, atol=1e-12)
+
+
+def test_pi_proportional_to_score_below_cap():
+    s = np.array([0.5, 0.25, 0.125, 0.0625, 0.03125, 0.03125], np.float32)  # exact in fp32
+    p, capped, r, R, q = pis(s, 2)
+    # 0.5 * 2 = 1 caps block 0; the rest share r = 1 in proportion to score
+    assert capped.tolist() == [True, False, False, False, False, False]
+    assert r == 1 and R == 1 << 31
+    assert p[1:] == [0.5, 0.25, 0.125, 0.0625, 0.0625]
+
+
+def test_zero_score_keeps_a_nonzero_chance_and_unit_score_caps():
+    s = np.zeros(10, np.float32)
+    s[0] = 1.0
+    q = oracle.quantised_scores(s)
+    assert q[0] == 1 << 32 and q[1:] == [1] * 9
+    p, capped, _, _, _ = pis(s, 3)
+    assert capped[0] and all(0 < x < 1 for x in p[1:])
+    assert abs(sum(p) - 3) < 1e-12
+
+
+def test_splitmix64_published_outputs():
+    with open(os.path.join(GOLDEN, "splitmix64_reference.json")) as f:
+        g = json.load(f)
+    gamma = int(g["gamma"], 16)
+    got = [oracle.splitmix64_mix((k * gamma) % 2**64) for k in (1, 2, 3)]
+    assert got == [int(x, 16) for x in g["outputs_from_state_0"]]
+
+
+def test_draw_is_second_mix_of_seed_xor_first():
+    # u = mix(mix(ctr + gamma) ^ seed) >> 32; with seed 0 and ctr 0 this is
+    # mix(first reference output) >> 32
+    first = 0xE220A8397B1DCDAF
+    assert oracle.draw_u32(0, 0) == oracle.splitmix64_mix(first) >> 32
+
+
+def test_sample_row_dense_short_circuit():
+    s = synthetic.random_scores(1, 64, 1)[0]
+    idx, lp, taken, r, R = oracle.sample_row(s, 64, seed=3, row=0, cap=64)
+    assert taken == 64 and idx.tolist() == list(range(64)) and np.all(lp == 0)
+    assert (r, R) == (0, 0)
+
+
+def test_sample_row_structure_and_log_pi():
+    nkb, n = 2000, 150
+    s = synthetic.random_scores(1, nkb, 11)[0]
+    p, capped, r, R, q = pis(s, n)
+    cap = oracle.plan_capacity(n, nkb)
+    idx, lp, taken, r2, R2 = oracle.sample_row(s, n, seed=5, row=7, cap=cap)
+    assert (r2, R2) == (r, R)
+    assert taken == len(idx) <= cap
+    assert np.all(np.diff(idx) > 0)                    # ascending, no repeats
+    assert all(capped[j] for j in np.flatnonzero(capped)) and set(np.flatnonzero(capped)) <= set(idx)
+    for j, l in zip(idx, lp):
+        if capped[j]:
+            assert l == 0.0
+        else:
+            assert l < 0 and abs(float(l) - math.log(p[j])) <= 2 * np.spacing(np.float32(abs(l)))
+
+
+def test_sample_row_draw_rule():
+    nkb, n, seed, row = 300, 30, 9, 123
+    s = synthetic.random_scores(1, nkb, 12)[0]
+    _, capped, r, R, q = pis(s, n)
+    idx, _, _, _, _ = oracle.sample_row(s, n, seed, row, cap=nkb)
+    expect = [j for j in range(nkb)
+              if capped[j] or oracle.draw_u32(seed, row * nkb + j) * R < (r * q[j]) << 32]
+    assert idx.tolist() == expect
+
+
+def test_inclusion_frequencies_match_pi():
+    """Over 10^4 seeds each block's inclusion frequency is within 5 sigma of pi."""
+    nkb, n, S = 64, 10, 10000
+    s = synthetic.random_scores(1, nkb, 21)[0]
+    p, _, _, _, _ = pis(s, n)
+    p = np.array(p)
+    hits = np.zeros(nkb)
+    sizes = np.zeros(S)
+    for seed in range(S):
+        idx, _, taken, _, _ = oracle.sample_row(s, n, seed, 0, cap=nkb)
+        hits[idx] += 1
+        sizes[seed] = taken
+    freq = hits / S
+    sigma = np.sqrt(p * (1 - p) / S) + 1e-12
+    assert np.all(np.abs(freq - p) <= 5 * sigma + 1e-12)
+    var = float((p * (1 - p)).sum())
+    assert abs(sizes.mean() - n) <= 5 * math.sqrt(var / S)
+
+
+def test_plan_capacity_formula():
+    assert oracle.plan_capacity(819, 8190) == 1088
+    assert oracle.plan_capacity(13, 128) == 96
+    assert oracle.plan_capacity(8190, 8190) == 8190
+    assert oracle.plan_capacity(1512, 18900) == 1856   # 1512 + ceil(311.07) + 32
+    assert oracle.plan_capacity(2376, 29700) == 2816   # 2376 + 390 + 32 = 2798 -> 2816
