@@ -1,0 +1,381 @@
+"""Benchmark of the AB-Attention hot path on B200.
+
+One step = one attention call of a Wan2.1-14B-shaped 480p self-attention layer
+(B=1, 40 heads, d=128, 21x30x52 = 32760 tokens, budget 819 of 8190 key blocks):
+IBCS selector (pool, k-means, score) + SIP sampler + HT sparse attention, all
+in libabsa.so.  Metric: ms per attention call (lower is better), with the
+effective TFLOP/s of the sparse attention beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (under torchrun): every rank runs the same layer on its own GPU
+(independent replicas, no collective on the data path); the time is the max
+over ranks and the value is ms per call over all N*K calls.
+--impl reference times the CPU oracle (plain C, OpenMP) on a bounded sample of
+the same layer and extrapolates to ms per call.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per attention call (select+sample+sparse attn) at 1 B200; effective TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target wall time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload():
+    from block_sparse_attention_selector_b200 import synthetic
+
+    return synthetic.WAN480
+
+
+def config_of(w, extra=None):
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+           "grid": [w.T, w.Hg, w.Wg], "budget_blocks": w.budget, "kv_blocks": w.nkb,
+           "query_blocks": w.nqb, "inputs": "seeded synthetic Fourier-feature q/k, Gaussian v",
+           "l2": "flushed before every timed step (256 MiB write, outside the step events); "
+                 "inputs (1 GiB q/k/v) are also larger than L2"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w, q, k, v, n_qb, seed=1):
+    """Run the oracle hot path on query blocks [0, n_qb) of every head; seconds."""
+    import oracle
+
+    t0 = time.perf_counter()
+    scores, _, _, _ = oracle.select_scores(q, k, qb_range=(0, n_qb))
+    sub = np.ascontiguousarray(scores[:, :, :n_qb])
+    cap = oracle.plan_capacity(w.budget, w.nkb)
+    plan = oracle.sample_plan(sub, w.budget, seed, cap)
+    full = dict(counts=np.zeros((w.B, w.H, w.nqb), np.int32),
+                kv_index=np.zeros((w.B, w.H, w.nqb, cap), np.int32),
+                log_pi=np.zeros((w.B, w.H, w.nqb, cap), np.float32))
+    full["counts"][:, :, :n_qb] = plan["counts"]
+    full["kv_index"][:, :, :n_qb] = plan["kv_index"]
+    full["log_pi"][:, :, :n_qb] = plan["log_pi"]
+    oracle.sparse_attention(q, k, v, full, qb_range=(0, n_qb))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, q, k, v, target_s):
+    import oracle
+
+    t1 = oracle_sample(w, q, k, v, 1)
+    n_qb = int(max(1, min(w.nqb, math.floor(target_s / max(t1, 1e-3)))))
+    t = oracle_sample(w, q, k, v, n_qb) if n_qb > 1 else t1
+    ms = t * 1e3 * w.nqb / n_qb
+    return {"value": ms, "unit": "ms", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"query blocks 0..{n_qb - 1} of all {w.H} heads ({n_qb * w.H} of "
+                      f"{w.nqb * w.H} plan rows: select+sample+attention), wall {t:.1f} s, "
+                      f"extrapolated x{w.nqb / n_qb:.1f} to the full layer"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_sparse_attention_selector_b200 import synthetic
+
+    w = workload()
+    q, k, v = synthetic.layer_qkv_bits(w)
+    import oracle
+
+    oracle.lib()
+    steps = max(1, args.steps)
+    per_step_target = max(1.0, min(args.cpu_seconds, 120.0 / (steps + args.warmup)))
+    t1 = oracle_sample(w, q, k, v, 1)
+    n_qb = int(max(1, min(w.nqb, math.floor(per_step_target / max(t1, 1e-3)))))
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, n_qb)
+    times = [oracle_sample(w, q, k, v, n_qb) for _ in range(steps)]
+    ms = float(np.mean(times)) * 1e3 * w.nqb / n_qb
+    sample = (f"each step: query blocks 0..{n_qb - 1} of all {w.H} heads "
+              f"(select+sample+attention), extrapolated x{w.nqb / n_qb:.1f}")
+    line = {"impl": "reference", "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": ms, "unit": "ms", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"absa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops", 1590.0), d.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def recorded_traffic(kernel_src):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    with open(kernel_src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    ent = rec.get("sparse_attention")
+    if ent and ent.get("source_sha256_16") == digest:
+        return ent.get("dram_bytes_per_launch")
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_selector_b200 as absa
+    from block_sparse_attention_selector_b200 import synthetic
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    w = workload()
+    q_bits, k_bits, v_bits = synthetic.layer_qkv_bits(w)
+
+    def to_dev(b):
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q, k, v = to_dev(q_bits), to_dev(k_bits), to_dev(v_bits)
+    p = absa.params_for(w, seed=1234 + rank)
+    plan = absa.Plan(p, dev)
+    scores = torch.empty((w.B, w.H, w.nqb, w.nkb), dtype=torch.float32, device=dev)
+    ws = absa.workspace(p, dev)
+    o = torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        absa.select_scores(p, q, k, scores, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        absa.sample_plan(p, scores, plan)
+        if ev is not None:
+            ev[2].record(stream)
+        absa.sparse_attention(p, q, k, v, plan, o)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    plan.check()
+
+    K = args.steps
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    attn_flops = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        for i in range(K):
+            flush.zero_()
+            step(events[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    plan.check()
+    counts = plan.counts.to(torch.int64).cpu().numpy()
+    nvalid = np.full(w.nqb, 128, np.int64)
+    nvalid[-1] = w.last_valid
+    # algorithmic flops of the sparse attention: 4 d per (query row, key token)
+    flops = float(4 * w.d * (counts * 4 * nvalid[None, None, :]).sum())
+    attn_flops = flops
+    sel = np.array([e[0].elapsed_time(e[1]) for e in events])
+    smp = np.array([e[1].elapsed_time(e[2]) for e in events])
+    att = np.array([e[2].elapsed_time(e[3]) for e in events])
+    tot = sel + smp + att
+    t_local = float(tot.sum())
+    t = torch.tensor([t_local], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t_max = float(t.item())
+    ms_per_call = t_max / (K * world)
+
+    # dense reference kernel on the same shapes (companion number)
+    ev_d = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    dense_ms = []
+    for _ in range(3):
+        flush.zero_()
+        ev_d[0].record(stream)
+        absa.dense_reference(p, q, k, v, o)
+        ev_d[1].record(stream)
+        torch.cuda.synchronize()
+        dense_ms.append(ev_d[0].elapsed_time(ev_d[1]))
+
+    # end to end through the public API with host buffers
+    q_h, k_h, v_h = (torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for b in (q_bits, k_bits, v_bits))
+    o_h = torch.empty_like(q_h).pin_memory()
+    e2e = []
+    for i in range(1 + args.e2e_steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        absa.select_plan(p, q, k, plan, scores, ws)
+        absa.sparse_attention(p, q, k, v, plan, o)
+        o_h.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            e2e.append(e0.elapsed_time(e1))
+    te = torch.tensor([float(np.sum(e2e))], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / (len(e2e) * world)
+
+    peak_tf, hbm_gbs, peak_src = measured_peaks()
+    att_ms = float(att.mean())
+    achieved_tf = attn_flops / (att_ms * 1e-3) / 1e12
+    sel_bytes = 2 * q.numel() * 2  # algorithmic: read q and k once
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": ms_per_call, "unit": "ms", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": t_max / K, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, {
+                "parallelism": f"replicas{world}" if world > 1 else "single",
+                "tflops_effective": attn_flops / (float(tot.mean()) * 1e-3) / 1e12,
+                "attention_tflops": achieved_tf,
+                "breakdown_ms": {"select_scores": float(sel.mean()), "sample": float(smp.mean()),
+                                 "sparse_attention": att_ms},
+                "plan_reuse_ms_per_call": float(sel.mean() + smp.mean()) / 4 + att_ms,
+                "dense_reference_ms": float(np.median(dense_ms)),
+                "dense_tflops": 4.0 * w.d * w.N * w.N * w.B * w.H / (np.median(dense_ms) * 1e-3) / 1e12,
+                "mean_blocks_per_row": float(counts.mean()),
+                "selector_hbm_frac_of_measured": sel_bytes / (float(sel.mean()) * 1e-3) / 1e9 / hbm_gbs,
+            }),
+            "roofline": {"bound": "tensor", "kernel": "absa_attention_kernel<128,sparse>",
+                         "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved_tf / peak_tf, "peak_source": f"{peak_src} bf16 (burst)",
+                         "traffic": recorded_traffic(os.path.join(
+                             ROOT, "block_sparse_attention_selector_b200", "csrc", "attention.cu")),
+                         "algorithmic_flops_per_launch": attn_flops},
+            "e2e": {"value": e2e_ms, "unit": "ms",
+                    "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2},
+            "gpu_launches": 5 * K,
+            "clocks": clocks.summary(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w, q_bits, k_bits, v_bits, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

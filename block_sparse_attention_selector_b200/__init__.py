@@ -1,0 +1,160 @@
+"""AB-Attention block-sparse attention selector for B200 (sm_100a).
+
+The hot path -- IBCS selector, SIP sampler and Horvitz-Thompson sparse
+attention over 4-token key/value blocks, plus a dense attention kernel --
+lives in libabsa.so behind the C ABI of include/absa.h.  This package binds it
+with ctypes (``_abi``: the C names, raw device pointers) and offers a thin
+torch-facing layer below (device memory and streams come from PyTorch; every
+step of the computation runs in the library's CUDA kernels).
+"""
+import math
+
+from . import _abi
+from ._abi import (AbsaError, absa_check_params, absa_dense_reference, absa_params, absa_plan,
+                   absa_plan_capacity, absa_plan_check, absa_sample_plan, absa_select_plan,
+                   absa_select_scores, absa_sparse_attention, absa_workspace_bytes)
+from .synthetic import Workload
+
+__all__ = [
+    "AbsaError", "Plan", "Workload", "absa_check_params", "absa_dense_reference", "absa_params",
+    "absa_plan", "absa_plan_capacity", "absa_plan_check", "absa_sample_plan", "absa_select_plan",
+    "absa_select_scores", "absa_sparse_attention", "absa_workspace_bytes", "dense_reference",
+    "make_params", "sample_plan", "select_plan", "select_scores", "sparse_attention",
+    "workspace", "version",
+]
+
+
+def version():
+    return _abi.version()
+
+
+def make_params(B, H, N, d, T, Hg, Wg, budget_blocks, seed=0, softmax_scale=None,
+                kmeans_iters=3):
+    """An absa_params block (q_block 128, kv_block 4, 8 clusters)."""
+    p = absa_params()
+    p.B, p.H, p.N, p.d = int(B), int(H), int(N), int(d)
+    p.T, p.Hg, p.Wg = int(T), int(Hg), int(Wg)
+    p.q_block, p.kv_block, p.n_clusters = 128, 4, 8
+    p.kmeans_iters = int(kmeans_iters)
+    p.budget_blocks = int(budget_blocks)
+    p.seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    p.softmax_scale = float(1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale)
+    return p
+
+
+def params_for(w: Workload, seed=0, budget=None):
+    return make_params(w.B, w.H, w.N, w.d, w.T, w.Hg, w.Wg,
+                       w.budget if budget is None else budget, seed)
+
+
+def _stream_handle(stream):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_bf16(*ts):
+    import torch
+
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, o must be contiguous bf16 CUDA tensors [B,H,N,d]")
+
+
+class Plan:
+    """Device arrays of a SIP sampling plan (torch tensors) and their C view."""
+
+    def __init__(self, p, device="cuda", capacity=None):
+        import torch
+
+        cap = absa_plan_capacity(p) if capacity is None else int(capacity)
+        if cap < 1:
+            raise AbsaError(_abi.ABSA_ERR_INVALID_ARG, "absa_plan_capacity")
+        nqb, nkb = (p.N + 127) // 128, (p.N + 3) // 4
+        rows = (p.B, p.H, nqb)
+        self.capacity = cap
+        self.counts = torch.zeros(rows, dtype=torch.int32, device=device)
+        self.kv_index = torch.zeros(rows + (cap,), dtype=torch.int32, device=device)
+        self.log_pi = torch.zeros(rows + (cap,), dtype=torch.float32, device=device)
+        self.r_R = torch.zeros(rows + (2,), dtype=torch.int64, device=device)
+        self.status = torch.zeros(4, dtype=torch.int32, device=device)
+        self.c = absa_plan(nqb, nkb, cap, self.counts.data_ptr(), self.kv_index.data_ptr(),
+                           self.log_pi.data_ptr(), self.r_R.data_ptr(), self.status.data_ptr())
+
+    def check(self, stream=None):
+        """Synchronise and raise on a device-reported error (overflow, bad plan, timeout)."""
+        _abi.check(absa_plan_check(self.c, _stream_handle(stream)), "absa_plan_check")
+
+
+def workspace(p, device="cuda"):
+    import torch
+
+    n = absa_workspace_bytes(p)
+    if n == 0:
+        raise AbsaError(_abi.ABSA_ERR_INVALID_ARG, "absa_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def select_scores(p, q, k, scores=None, ws=None, stream=None):
+    import torch
+
+    _check_bf16(q, k)
+    nqb, nkb = (p.N + 127) // 128, (p.N + 3) // 4
+    if scores is None:
+        scores = torch.empty((p.B, p.H, nqb, nkb), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(p, q.device)
+    _abi.check(absa_select_scores(p, _ptr(q), _ptr(k), _ptr(scores), _ptr(ws), ws.numel(),
+                                  _stream_handle(stream)), "absa_select_scores")
+    return scores, ws
+
+
+def sample_plan(p, scores, plan=None, stream=None):
+    if plan is None:
+        plan = Plan(p, scores.device)
+    _abi.check(absa_sample_plan(p, _ptr(scores), plan.c, _stream_handle(stream)),
+               "absa_sample_plan")
+    return plan
+
+
+def select_plan(p, q, k, plan=None, scores=None, ws=None, stream=None):
+    import torch
+
+    _check_bf16(q, k)
+    nqb, nkb = (p.N + 127) // 128, (p.N + 3) // 4
+    if plan is None:
+        plan = Plan(p, q.device)
+    if scores is None:
+        scores = torch.empty((p.B, p.H, nqb, nkb), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(p, q.device)
+    _abi.check(absa_select_plan(p, _ptr(q), _ptr(k), _ptr(scores), plan.c, _ptr(ws), ws.numel(),
+                                _stream_handle(stream)), "absa_select_plan")
+    return plan, scores, ws
+
+
+def sparse_attention(p, q, k, v, plan, out=None, stream=None):
+    import torch
+
+    _check_bf16(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    _abi.check(absa_sparse_attention(p, _ptr(q), _ptr(k), _ptr(v), plan.c, _ptr(out),
+                                     _stream_handle(stream)), "absa_sparse_attention")
+    return out
+
+
+def dense_reference(p, q, k, v, out=None, status=None, stream=None):
+    import torch
+
+    _check_bf16(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    _abi.check(absa_dense_reference(p, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(status),
+                                    _stream_handle(stream)), "absa_dense_reference")
+    return out

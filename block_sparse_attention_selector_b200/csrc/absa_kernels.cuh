@@ -1,0 +1,40 @@
+// absa_kernels.cuh -- host-side launchers of the AB-Attention kernels (sm_100a).
+// Each kernel lives in its own translation unit; the C ABI (api.cu) validates
+// arguments and calls these.
+#pragma once
+
+#include "absa_device.cuh"
+
+namespace absa {
+
+constexpr int kSampleMaxKvBlocks = 49152;
+
+// K1: mean key of every 4-token block as bf16 hi + lo.
+cudaError_t launch_pool(const __nv_bfloat16 *k, __nv_bfloat16 *kbar_hi, __nv_bfloat16 *kbar_lo,
+                        int64_t BH, int N, int nkb, int d, cudaStream_t stream);
+
+// K2: per-query-block k-means (8 clusters), centroids, their bf16 split,
+// weights and final assignment.
+cudaError_t launch_kmeans(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int d, int iters,
+                          float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
+                          uint8_t *assign, cudaStream_t stream);
+
+// K3: block scores from the centroid split and the key-block split.
+cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,
+                         const CUtensorMap &tm_mu_hi, const CUtensorMap &tm_mu_lo, const float *w,
+                         float *scores, int64_t BH, int nqb, int nkb, int d, float softmax_scale,
+                         int32_t *status, cudaStream_t stream);
+
+// K4: SIP plan rows from a score array.
+cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
+                          int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
+                          uint64_t *r_R, int32_t *status, cudaStream_t stream);
+
+// K5 (dense = false) / K6 (dense = true): attention over 128-token tiles.
+cudaError_t launch_attention(bool dense, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                             const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N, int nqb,
+                             int nkb, int d, float softmax_scale, const int32_t *counts,
+                             const int32_t *kv_index, const float *log_pi, int cap,
+                             int32_t *status, cudaStream_t stream);
+
+}  // namespace absa

@@ -1,0 +1,295 @@
+// api.cu -- the C ABI declared in include/absa.h: argument validation,
+// workspace layout, tensor maps for the TMA loads, and kernel launches on the
+// caller's stream.  No allocation, no synchronisation (except absa_plan_check).
+#include <math.h>
+#include <mutex>
+
+#include "absa_kernels.cuh"
+
+using namespace absa;
+
+namespace {
+
+struct Dims {
+    int64_t BH;
+    int nqb, nkb;
+};
+
+Dims dims_of(const absa_params *p) {
+    Dims d;
+    d.BH = (int64_t)p->B * p->H;
+    d.nqb = (p->N + 127) / 128;
+    d.nkb = (p->N + 3) / 4;
+    return d;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct WsLayout {
+    size_t kbar_hi, kbar_lo, mu, mu_hi, mu_lo, w, assign, total;
+};
+
+WsLayout ws_layout(const absa_params *p) {
+    const Dims dm = dims_of(p);
+    const size_t d = (size_t)p->d;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) & ~(size_t)255;
+        return o;
+    };
+    WsLayout L;
+    L.kbar_hi = take((size_t)dm.BH * dm.nkb * d * 2);
+    L.kbar_lo = take((size_t)dm.BH * dm.nkb * d * 2);
+    L.mu = take((size_t)dm.BH * dm.nqb * 8 * d * 4);
+    L.mu_hi = take((size_t)dm.BH * dm.nqb * 8 * d * 2);
+    L.mu_lo = take((size_t)dm.BH * dm.nqb * 8 * d * 2);
+    L.w = take((size_t)dm.BH * dm.nqb * 8 * 4);
+    L.assign = take((size_t)dm.BH * dm.nqb * 128);
+    L.total = off;
+    return L;
+}
+
+absa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ABSA_OK : ABSA_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols fastest), box 64 x 128 with 128-byte swizzle.
+bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int cols) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), gdim, gstride,
+              box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+absa_status check_plan(const absa_params *p, const absa_plan *plan) {
+    if (!plan) return ABSA_ERR_INVALID_ARG;
+    const Dims dm = dims_of(p);
+    if (plan->n_qblocks != dm.nqb || plan->n_kvblocks != dm.nkb || plan->capacity < 1)
+        return ABSA_ERR_INVALID_ARG;
+    if (!plan->counts || !plan->kv_index || !plan->log_pi || !plan->r_R || !plan->status)
+        return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(plan->counts) || !aligned16(plan->kv_index) || !aligned16(plan->log_pi) ||
+        !aligned16(plan->r_R) || (reinterpret_cast<uintptr_t>(plan->status) & 3u))
+        return ABSA_ERR_INVALID_ARG;
+    if ((double)dm.BH * dm.nqb * (double)plan->capacity > 9.0e15) return ABSA_ERR_INVALID_ARG;
+    return ABSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *absa_version(void) { return "absa 0.1.0 (sm_100a)"; }
+
+const char *absa_status_string(absa_status s) {
+    switch (s) {
+        case ABSA_OK: return "ABSA_OK";
+        case ABSA_ERR_INVALID_ARG: return "ABSA_ERR_INVALID_ARG";
+        case ABSA_ERR_UNSUPPORTED: return "ABSA_ERR_UNSUPPORTED";
+        case ABSA_ERR_WORKSPACE: return "ABSA_ERR_WORKSPACE";
+        case ABSA_ERR_CUDA: return "ABSA_ERR_CUDA";
+        case ABSA_ERR_PLAN_OVERFLOW: return "ABSA_ERR_PLAN_OVERFLOW";
+        case ABSA_ERR_BAD_PLAN: return "ABSA_ERR_BAD_PLAN";
+        case ABSA_ERR_TIMEOUT: return "ABSA_ERR_TIMEOUT";
+    }
+    return "ABSA_ERR_UNKNOWN";
+}
+
+absa_status absa_check_params(const absa_params *p) {
+    if (!p) return ABSA_ERR_INVALID_ARG;
+    if (p->B < 1 || p->H < 1 || p->N < 1 || p->d < 1) return ABSA_ERR_INVALID_ARG;
+    if (p->T < 1 || p->Hg < 1 || p->Wg < 1 ||
+        (int64_t)p->T * p->Hg * p->Wg != (int64_t)p->N)
+        return ABSA_ERR_INVALID_ARG;
+    if (p->budget_blocks < 1 || p->kmeans_iters < 1 || p->kmeans_iters > 16)
+        return ABSA_ERR_INVALID_ARG;
+    if (!isfinite(p->softmax_scale)) return ABSA_ERR_INVALID_ARG;
+    if (p->q_block != 128 || p->kv_block != 4 || p->n_clusters != 8) return ABSA_ERR_UNSUPPORTED;
+    if (p->d != 64 && p->d != 128) return ABSA_ERR_UNSUPPORTED;
+    const Dims dm = dims_of(p);
+    // TMA row coordinates and per-CTA indices are 32-bit
+    if (dm.BH * dm.nkb >= (int64_t)1 << 31 || dm.BH * dm.nqb * 8 >= (int64_t)1 << 31)
+        return ABSA_ERR_UNSUPPORTED;
+    if (dm.nkb > kSampleMaxKvBlocks) return ABSA_ERR_UNSUPPORTED;
+    return ABSA_OK;
+}
+
+int32_t absa_plan_capacity(const absa_params *p) {
+    if (absa_check_params(p) != ABSA_OK) return -1;
+    const int64_t nkb = dims_of(p).nkb;
+    const int64_t n = p->budget_blocks;
+    if (n >= nkb) return (int32_t)nkb;
+    int64_t c = (int64_t)sqrt((double)(64 * n));
+    while (c * c < 64 * n) ++c;  // ceil(8 sqrt(n))
+    while (c > 0 && (c - 1) * (c - 1) >= 64 * n) --c;
+    int64_t cap = ((n + c + 32 + 31) / 32) * 32;
+    return (int32_t)(cap < nkb ? cap : nkb);
+}
+
+size_t absa_workspace_bytes(const absa_params *p) {
+    if (absa_check_params(p) != ABSA_OK) return 0;
+    return ws_layout(p).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+absa_status select_scores_impl(const absa_params *p, const void *q, const void *k, float *scores,
+                               void *ws, size_t ws_bytes, int32_t *status, void *stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (!q || !k || !scores || !ws) return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || !aligned16(ws))
+        return ABSA_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(p);
+    if (ws_bytes < L.total) return ABSA_ERR_WORKSPACE;
+    const Dims dm = dims_of(p);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    auto *kb_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_hi);
+    auto *kb_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_lo);
+    auto *mu = reinterpret_cast<float *>(w8 + L.mu);
+    auto *mu_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_hi);
+    auto *mu_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_lo);
+    auto *w = reinterpret_cast<float *>(w8 + L.w);
+    auto *assign = w8 + L.assign;
+
+    CUtensorMap tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo;
+    if (!make_map_bf16(&tm_kb_hi, kb_hi, dm.BH * dm.nkb, p->d) ||
+        !make_map_bf16(&tm_kb_lo, kb_lo, dm.BH * dm.nkb, p->d) ||
+        !make_map_bf16(&tm_mu_hi, mu_hi, dm.BH * dm.nqb * 8, p->d) ||
+        !make_map_bf16(&tm_mu_lo, mu_lo, dm.BH * dm.nqb * 8, p->d))
+        return ABSA_ERR_CUDA;
+
+    cudaError_t e = launch_pool(static_cast<const __nv_bfloat16 *>(k), kb_hi, kb_lo, dm.BH, p->N,
+                                dm.nkb, p->d, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = launch_kmeans(static_cast<const __nv_bfloat16 *>(q), dm.BH, p->N, dm.nqb, p->d,
+                      p->kmeans_iters, mu, mu_hi, mu_lo, w, assign, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, scores, dm.BH, dm.nqb, dm.nkb,
+                     p->d, p->softmax_scale, status, s);
+    return from_cuda(e);
+}
+
+absa_status sample_plan_impl(const absa_params *p, const float *scores, const absa_plan *plan,
+                             bool reset_status, void *stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (!scores || !aligned16(scores)) return ABSA_ERR_INVALID_ARG;
+    st = check_plan(p, plan);
+    if (st != ABSA_OK) return st;
+    const Dims dm = dims_of(p);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (reset_status) {
+        e = cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    e = launch_sample(scores, dm.BH * dm.nqb, dm.nkb, p->budget_blocks, p->seed, plan->capacity,
+                      plan->counts, plan->kv_index, plan->log_pi, plan->r_R, plan->status, s);
+    return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+absa_status absa_select_scores(const absa_params *p, const void *q, const void *k, float *scores,
+                               void *ws, size_t ws_bytes, void *stream) {
+    return select_scores_impl(p, q, k, scores, ws, ws_bytes, nullptr, stream);
+}
+
+absa_status absa_sample_plan(const absa_params *p, const float *scores, const absa_plan *plan,
+                             void *stream) {
+    return sample_plan_impl(p, scores, plan, true, stream);
+}
+
+absa_status absa_select_plan(const absa_params *p, const void *q, const void *k, float *scores,
+                             const absa_plan *plan, void *ws, size_t ws_bytes, void *stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    st = check_plan(p, plan);
+    if (st != ABSA_OK) return st;
+    if (cudaMemsetAsync(plan->status, 0, sizeof(int32_t),
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ABSA_ERR_CUDA;
+    st = select_scores_impl(p, q, k, scores, ws, ws_bytes, plan->status, stream);
+    if (st != ABSA_OK) return st;
+    return sample_plan_impl(p, scores, plan, false, stream);
+}
+
+absa_status absa_sparse_attention(const absa_params *p, const void *q, const void *k,
+                                  const void *v, const absa_plan *plan, void *o, void *stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    st = check_plan(p, plan);
+    if (st != ABSA_OK) return st;
+    if (!q || !k || !v || !o) return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return ABSA_ERR_INVALID_ARG;
+    const Dims dm = dims_of(p);
+    return from_cuda(launch_attention(
+        false, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), dm.BH, p->N,
+        dm.nqb, dm.nkb, p->d, p->softmax_scale, plan->counts, plan->kv_index, plan->log_pi,
+        plan->capacity, plan->status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,
+                                 const void *v, void *o, int32_t *status, void *stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (!q || !k || !v || !o) return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return ABSA_ERR_INVALID_ARG;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return ABSA_ERR_INVALID_ARG;
+    const Dims dm = dims_of(p);
+    return from_cuda(launch_attention(
+        true, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), dm.BH, p->N,
+        dm.nqb, dm.nkb, p->d, p->softmax_scale, nullptr, nullptr, nullptr, 0, status,
+        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+absa_status absa_plan_check(const absa_plan *plan, void *stream) {
+    if (!plan || !plan->status) return ABSA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return ABSA_ERR_CUDA;
+    int32_t flags = 0;
+    e = cudaMemcpy(&flags, plan->status, sizeof(flags), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return ABSA_ERR_CUDA;
+    if (flags & ABSA_DEVFLAG_TIMEOUT) return ABSA_ERR_TIMEOUT;
+    if (flags & ABSA_DEVFLAG_BAD_PLAN) return ABSA_ERR_BAD_PLAN;
+    if (flags & ABSA_DEVFLAG_OVERFLOW) return ABSA_ERR_PLAN_OVERFLOW;
+    return ABSA_OK;
+}
+
+}  // extern "C"

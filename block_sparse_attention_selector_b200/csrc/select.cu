@@ -1,0 +1,466 @@
+// select.cu -- IBCS block selector on sm_100a (AB-Attention summary page,
+// "AB-Attention's three techniques", IBCS paragraph):
+//   K1 absa_pool_kernel    mean key of every 4-token block, split hi+lo bf16
+//   K2 absa_kmeans_kernel  per-128-query-block Lloyd k-means in shared memory
+//   K3 absa_score_kernel   weighted centroid softmax over all key blocks, on
+//                          tcgen05 tensor cores (3-product bf16 split, TMEM)
+#include "absa_kernels.cuh"
+
+namespace absa {
+
+// ------------------------------------------------------------------------ K1
+
+// One thread per (row = (b,h,j), 8-element chunk): reads the 4 token rows of
+// block j (16-byte loads, a warp covers whole rows), averages in fp32 and
+// stores mean = hi + lo with hi = bf16(mean), lo = bf16(mean - hi).
+__global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__restrict__ k,
+                                                        __nv_bfloat16 *__restrict__ kbar_hi,
+                                                        __nv_bfloat16 *__restrict__ kbar_lo,
+                                                        int64_t BH, int N, int nkb, int d) {
+    const int ch = d >> 3;
+    const int64_t total = BH * (int64_t)nkb * ch;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int c = (int)(i % ch);
+        const int64_t row = i / ch;
+        const int64_t bh = row / nkb;
+        const int j = (int)(row % nkb);
+        const int t0 = 4 * j;
+        const int nt = min(4, N - t0);
+        const __nv_bfloat16 *src = k + ((bh * N + t0) * (int64_t)d) + c * 8;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int t = 0; t < nt; ++t) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)t * d));
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float2 f = __bfloat1622float2(h2[e]);
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
+            }
+        }
+        uint4 hi_u, lo_u;
+        uint32_t *hp = reinterpret_cast<uint32_t *>(&hi_u);
+        uint32_t *lp = reinterpret_cast<uint32_t *>(&lo_u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float m0 = nt == 4 ? acc[2 * e] * 0.25f : __fdiv_rn(acc[2 * e], (float)nt);
+            float m1 = nt == 4 ? acc[2 * e + 1] * 0.25f : __fdiv_rn(acc[2 * e + 1], (float)nt);
+            __nv_bfloat16 h0 = __float2bfloat16_rn(m0), h1 = __float2bfloat16_rn(m1);
+            __nv_bfloat16 l0 = __float2bfloat16_rn(m0 - __bfloat162float(h0));
+            __nv_bfloat16 l1 = __float2bfloat16_rn(m1 - __bfloat162float(h1));
+            hp[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+            lp[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        *reinterpret_cast<uint4 *>(kbar_hi + row * d + c * 8) = hi_u;
+        *reinterpret_cast<uint4 *>(kbar_lo + row * d + c * 8) = lo_u;
+    }
+}
+
+// ------------------------------------------------------------------------ K2
+
+// One CTA (128 threads) per query block.  The block's m valid queries are
+// widened to fp32 in shared memory (rows padded to D+1 words so that thread i
+// reading row i is bank-conflict free).  fp32 arithmetic in a fixed order:
+//  assignment (thread i): dist_c = sum over ascending e of fma(x-mu, x-mu, .),
+//                         argmin with ties to the lowest c;
+//  update     (thread e): member sums over ascending i, mu = sum / count
+//                         (IEEE division); an empty cluster keeps mu.
+template <int D>
+__global__ void __launch_bounds__(128) absa_kmeans_kernel(
+    const __nv_bfloat16 *__restrict__ q, int N, int nqb, int iters, float *__restrict__ mu_out,
+    __nv_bfloat16 *__restrict__ mu_hi, __nv_bfloat16 *__restrict__ mu_lo, float *__restrict__ w_out,
+    uint8_t *__restrict__ assign_out) {
+    constexpr int NC = 8;
+    constexpr int XS = D + 1;
+    extern __shared__ __align__(16) float kms[];
+    float *xs = kms;                    // [128][D+1]
+    float *mut = kms + 128 * XS;        // [D][8] centroids, transposed
+    int *asg = reinterpret_cast<int *>(mut + D * NC);  // [128]
+    int *cnt_s = asg + 128;             // [8]
+
+    const int tid = threadIdx.x;
+    const int64_t row = blockIdx.x;     // (b*H + h)*nqb + qb
+    const int64_t bh = row / nqb;
+    const int qb = (int)(row % nqb);
+    const int m = min(128, N - qb * 128);
+    const __nv_bfloat16 *src = q + (bh * N + (int64_t)qb * 128) * D;
+
+    constexpr int CH = D / 8;
+    for (int idx = tid; idx < m * CH; idx += 128) {
+        const int r = idx / CH, c = idx % CH;
+        uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)r * D + c * 8));
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(h2[e]);
+            xs[r * XS + c * 8 + 2 * e] = f.x;
+            xs[r * XS + c * 8 + 2 * e + 1] = f.y;
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < NC * D; idx += 128) {
+        const int c = idx / D, e = idx % D;
+        mut[e * NC + c] = xs[((c * m) / NC) * XS + e];
+    }
+    __syncthreads();
+
+    int cnt[NC];
+    for (int it = 0; it < iters; ++it) {
+        if (tid < m) {
+            float dist[NC];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) dist[c] = 0.f;
+            const float *xr = xs + tid * XS;
+#pragma unroll 4
+            for (int e = 0; e < D; ++e) {
+                const float xe = xr[e];
+                const float4 m0 = *reinterpret_cast<const float4 *>(mut + e * NC);
+                const float4 m1 = *reinterpret_cast<const float4 *>(mut + e * NC + 4);
+                const float mc[NC] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    const float diff = __fsub_rn(xe, mc[c]);
+                    dist[c] = __fmaf_rn(diff, diff, dist[c]);
+                }
+            }
+            int best = 0;
+            float bd = dist[0];
+#pragma unroll
+            for (int c = 1; c < NC; ++c)
+                if (dist[c] < bd) {
+                    bd = dist[c];
+                    best = c;
+                }
+            asg[tid] = best;
+        }
+        __syncthreads();
+        {
+            float acc[NC];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                acc[c] = 0.f;
+                cnt[c] = 0;
+            }
+            const int e = tid < D ? tid : 0;
+            for (int i = 0; i < m; ++i) {
+                const int a = asg[i];
+                const float xv = xs[i * XS + e];
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+                    if (a == c) {
+                        acc[c] = __fadd_rn(acc[c], xv);
+                        cnt[c] += 1;
+                    }
+            }
+            if (tid < D) {
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+                    if (cnt[c] > 0) mut[tid * NC + c] = __fdiv_rn(acc[c], (float)cnt[c]);
+            }
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) cnt_s[c] = cnt[c];
+    }
+    __syncthreads();
+    if (tid < NC) w_out[row * NC + tid] = __fdiv_rn((float)cnt_s[tid], (float)m);
+    for (int idx = tid; idx < NC * D; idx += 128) {
+        const int c = idx / D, e = idx % D;
+        const float v = mut[e * NC + c];
+        const int64_t o = (row * NC + c) * D + e;
+        mu_out[o] = v;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        mu_hi[o] = h;
+        mu_lo[o] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+    assign_out[row * 128 + tid] = tid < m ? (uint8_t)asg[tid] : (uint8_t)255;
+}
+
+// ------------------------------------------------------------------------ K3
+
+// One CTA per (b, h, group of 16 query blocks); the group's 128 centroid rows
+// (16 blocks x 8 clusters) stay in shared memory while tiles of 128 key blocks
+// stream through a 2-stage TMA ring.  Logits are mu . kbar computed as
+// hi*hi + hi*lo + lo*hi with three bf16 tcgen05 MMAs per k-step (error about
+// 2^-16 relative, far below the score tolerance).
+//   pass 1: D[(qb,c), j] = mu . kbar   (A = centroids, B = key tile); the
+//           thread owning TMEM lane (qb,c) keeps an online max and sum of
+//           exp2 over j and ends with L = lse2 - log2(w) for its centroid;
+//   pass 2: D[j, (qb,c)] = kbar . mu   (A = key tile, B = centroids); the
+//           thread owning lane j forms s_j = sum_c exp2(scaled logit - L_c)
+//           for each of the 16 query blocks and stores it.
+// Warps: 0 TMA producer, 1 MMA issuer (+TMEM owner), 2..5 epilogue.
+template <int D>
+struct ScoreSmem {
+    static constexpr int kRegions = D / 64;                 // 64-element SW128 regions
+    static constexpr int kTile = 128 * 128;                 // one region of 128 rows (bytes)
+    static constexpr int kMuBytes = 2 * kRegions * kTile;   // hi + lo
+    static constexpr int kKbBytes = 2 * kRegions * kTile;   // one stage, hi + lo
+    static constexpr int kMuOff = 0;
+    static constexpr int kKbOff = kMuBytes;
+    static constexpr int kLOff = kKbOff + 2 * kKbBytes;
+    static constexpr int kBarOff = kLOff + 128 * 4;
+    static constexpr int kBytes = kBarOff + 16 * 8 + 16;
+    static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) absa_score_kernel(
+    const __grid_constant__ CUtensorMap tm_kb_hi, const __grid_constant__ CUtensorMap tm_kb_lo,
+    const __grid_constant__ CUtensorMap tm_mu_hi, const __grid_constant__ CUtensorMap tm_mu_lo,
+    const float *__restrict__ w, float *__restrict__ scores, int nqb, int nkb, int groups,
+    float scale_log2, int32_t *status) {
+    using S = ScoreSmem<D>;
+    extern __shared__ uint8_t score_smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(score_smem_raw) + 1023) & ~uintptr_t(1023));
+    float *Ltab = reinterpret_cast<float *>(sm + S::kLOff);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::kBarOff);
+    uint64_t *mu_full = bars + 0;
+    uint64_t *kb_full = bars + 1;   // [2]
+    uint64_t *kb_empty = bars + 3;  // [2]
+    uint64_t *d_full = bars + 5;    // [2]
+    uint64_t *d_empty = bars + 7;   // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 10);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t bh = blockIdx.x / groups;
+    const int qb0 = (blockIdx.x % groups) * 16;
+    const int T = (nkb + 127) / 128;
+    const int64_t kv_row0 = bh * nkb;
+    const int64_t mu_row0 = (bh * nqb + qb0) * 8;
+
+    if (threadIdx.x == 0) {
+        mbar_init(mu_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(kb_full + s, 1);
+            mbar_init(kb_empty + s, 1);
+            mbar_init(d_full + s, 1);
+            mbar_init(d_empty + s, 4);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_kb_hi);
+            tma_prefetch_desc(&tm_kb_lo);
+            mbar_arrive_expect_tx(mu_full, S::kMuBytes);
+            const uint32_t mu_base = smem_u32(sm + S::kMuOff);
+            for (int r = 0; r < S::kRegions; ++r) {
+                tma_load_2d(mu_base + r * S::kTile, &tm_mu_hi, 64 * r, (int)mu_row0, mu_full);
+                tma_load_2d(mu_base + (S::kRegions + r) * S::kTile, &tm_mu_lo, 64 * r,
+                            (int)mu_row0, mu_full);
+            }
+            for (int g = 0; g < 2 * T; ++g) {
+                const int st = g & 1;
+                const int t = g % T;
+                if (g >= 2 && !mbar_wait(kb_empty + st, ((g - 2) >> 1) & 1, status, abort_flag))
+                    break;
+                mbar_arrive_expect_tx(kb_full + st, S::kKbBytes);
+                const uint32_t kb_base = smem_u32(sm + S::kKbOff + st * S::kKbBytes);
+                const int y = (int)(kv_row0 + (int64_t)t * 128);
+                for (int r = 0; r < S::kRegions; ++r) {
+                    tma_load_2d(kb_base + r * S::kTile, &tm_kb_hi, 64 * r, y, kb_full + st);
+                    tma_load_2d(kb_base + (S::kRegions + r) * S::kTile, &tm_kb_lo, 64 * r, y,
+                                kb_full + st);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0);
+            const uint32_t mu_base = smem_u32(sm + S::kMuOff);
+            bool ok = mbar_wait(mu_full, 0, status, abort_flag);
+            for (int g = 0; ok && g < 2 * T; ++g) {
+                const int st = g & 1;
+                const int buf = g & 1;
+                const bool pass2 = g >= T;
+                if (!mbar_wait(kb_full + st, (g >> 1) & 1, status, abort_flag)) break;
+                if (g >= 2 && !mbar_wait(d_empty + buf, ((g - 2) >> 1) & 1, status, abort_flag))
+                    break;
+                tc_fence_after();
+                const uint32_t kb_base = smem_u32(sm + S::kKbOff + st * S::kKbBytes);
+                const uint32_t a_base = pass2 ? kb_base : mu_base;
+                const uint32_t b_base = pass2 ? mu_base : kb_base;
+                const uint32_t dt = tmem + buf * 128;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
+                    const uint32_t lo = S::kRegions * S::kTile;
+                    const uint64_t ah = sw128_desc(a_base + off, 16, 1024);
+                    const uint64_t al = sw128_desc(a_base + lo + off, 16, 1024);
+                    const uint64_t bhd = sw128_desc(b_base + off, 16, 1024);
+                    const uint64_t bl = sw128_desc(b_base + lo + off, 16, 1024);
+                    tc_mma_f16(dt, ah, bhd, idesc, ks > 0);
+                    tc_mma_f16(dt, ah, bl, idesc, 1);
+                    tc_mma_f16(dt, al, bhd, idesc, 1);
+                }
+                tc_commit(d_full + buf);
+                tc_commit(kb_empty + st);
+            }
+        }
+    } else {
+        // epilogue: thread <-> TMEM lane (warps 2..5 own lane quarters 2,3,0,1)
+        const int quarter = warp & 3;
+        const int lrow = quarter * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+        bool ok = true;
+        // pass 1: online log-sum-exp over the key blocks of this centroid row
+        float mx = -INFINITY, sum = 0.f;
+        for (int t = 0; t < T && ok; ++t) {
+            const int buf = t & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(d_full + buf, (t >> 1) & 1, status, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[4][32];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(d_empty + buf);
+            const int ncols = min(128, nkb - t * 128);
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (ch * 32 + i < ncols) tmax = fmaxf(tmax, __uint_as_float(v[ch][i]));
+            if (tmax > mx) {
+                sum *= ex2((mx - tmax) * scale_log2);
+                mx = tmax;
+            }
+            const float moff = -mx * scale_log2;
+            float acc = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (ch * 32 + i < ncols)
+                        acc += ex2(__fmaf_rn(__uint_as_float(v[ch][i]), scale_log2, moff));
+            sum += acc;
+        }
+        {
+            const int qb = qb0 + (lrow >> 3);
+            const float wc = qb < nqb ? w[(bh * nqb + qb) * 8 + (lrow & 7)] : 0.f;
+            const float lse2 = mx * scale_log2 + log2f(sum);
+            Ltab[lrow] = wc > 0.f ? lse2 - log2f(wc) : INFINITY;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // pass 2: combine the 8 centroids of each query block for key block j = lane row
+        for (int t = 0; t < T && ok; ++t) {
+            const int g = T + t;
+            const int buf = g & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(d_full + buf, (g >> 1) & 1, status, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[4][32];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(d_empty + buf);
+            const int j = t * 128 + lrow;
+            if (j < nkb) {
+#pragma unroll
+                for (int qbl = 0; qbl < 16; ++qbl) {
+                    const int qb = qb0 + qbl;
+                    if (qb >= nqb) continue;
+                    const float4 L0 = *reinterpret_cast<const float4 *>(Ltab + qbl * 8);
+                    const float4 L1 = *reinterpret_cast<const float4 *>(Ltab + qbl * 8 + 4);
+                    const float Lc[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
+                    float s = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int col = qbl * 8 + c;
+                        s += ex2(__fmaf_rn(__uint_as_float(v[col >> 5][col & 31]), scale_log2,
+                                           -Lc[c]));
+                    }
+                    scores[(bh * nqb + qb) * (int64_t)nkb + j] = s;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+
+cudaError_t launch_pool(const __nv_bfloat16 *k, __nv_bfloat16 *kbar_hi, __nv_bfloat16 *kbar_lo,
+                        int64_t BH, int N, int nkb, int d, cudaStream_t stream) {
+    const int64_t total = BH * (int64_t)nkb * (d / 8);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    absa_pool_kernel<<<(unsigned)blocks, 256, 0, stream>>>(k, kbar_hi, kbar_lo, BH, N, nkb, d);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int iters,
+                                   float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
+                                   uint8_t *assign, cudaStream_t stream) {
+    const int smem = (128 * (D + 1) + D * 8) * 4 + 136 * 4;
+    cudaError_t e = cudaFuncSetAttribute(absa_kmeans_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    absa_kmeans_kernel<D><<<(unsigned)(BH * nqb), 128, smem, stream>>>(q, N, nqb, iters, mu, mu_hi,
+                                                                      mu_lo, w, assign);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kmeans(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int d, int iters,
+                          float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
+                          uint8_t *assign, cudaStream_t stream) {
+    return d == 64 ? launch_kmeans_d<64>(q, BH, N, nqb, iters, mu, mu_hi, mu_lo, w, assign, stream)
+                   : launch_kmeans_d<128>(q, BH, N, nqb, iters, mu, mu_hi, mu_lo, w, assign, stream);
+}
+
+template <int D>
+static cudaError_t launch_score_d(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c,
+                                  const CUtensorMap &dd, const float *w, float *scores, int64_t BH,
+                                  int nqb, int nkb, float scale_log2, int32_t *status,
+                                  cudaStream_t stream) {
+    const int smem = ScoreSmem<D>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(absa_score_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int groups = (nqb + 15) / 16;
+    absa_score_kernel<D><<<(unsigned)(BH * groups), 192, smem, stream>>>(
+        a, b, c, dd, w, scores, nqb, nkb, groups, scale_log2, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,
+                         const CUtensorMap &tm_mu_hi, const CUtensorMap &tm_mu_lo, const float *w,
+                         float *scores, int64_t BH, int nqb, int nkb, int d, float softmax_scale,
+                         int32_t *status, cudaStream_t stream) {
+    const float scale_log2 = softmax_scale * 1.4426950408889634f;
+    return d == 64 ? launch_score_d<64>(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, scores, BH,
+                                        nqb, nkb, scale_log2, status, stream)
+                   : launch_score_d<128>(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, scores, BH,
+                                         nqb, nkb, scale_log2, status, stream);
+}
+
+}  // namespace absa

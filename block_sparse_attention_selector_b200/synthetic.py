@@ -86,11 +86,14 @@ def grid_coords(T: int, Hg: int, Wg: int) -> np.ndarray:
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round fp64 -> fp32 -> bf16 (each to nearest even); return uint16 bit patterns."""
     f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = f.view(np.uint32)
+    bias = (u >> np.uint32(16)) & np.uint32(1)
+    bias += np.uint32(0x7FFF)
+    bias += u                      # no overflow for finite values
+    out = (bias >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(f)
-    out = rounded.astype(np.uint16)
-    out[nan] = 0x7FC0
+    if nan.any():
+        out[nan] = 0x7FC0
     return out
 
 
@@ -110,20 +113,37 @@ def head_qkv(w: Workload, b: int, h: int, coords: np.ndarray | None = None):
     return q, k, v
 
 
-def layer_qkv_bits(w: Workload, heads: range | None = None):
-    """bf16 bit patterns of q, k, v: uint16 arrays [B, len(heads), N, d]."""
+def layer_qkv_bits(w: Workload, heads: range | None = None, threads: int | None = None):
+    """bf16 bit patterns of q, k, v: uint16 arrays [B, len(heads), N, d].
+
+    Heads are generated independently (each from its own seeded stream), in a
+    thread pool when there are several.
+    """
+    import concurrent.futures
+    import os
+
     heads = range(w.H) if heads is None else heads
     coords = grid_coords(w.T, w.Hg, w.Wg)
     shape = (w.B, len(heads), w.N, w.d)
     q = np.empty(shape, np.uint16)
     k = np.empty(shape, np.uint16)
     v = np.empty(shape, np.uint16)
-    for b in range(w.B):
-        for i, h in enumerate(heads):
-            qh, kh, vh = head_qkv(w, b, h, coords)
-            q[b, i] = to_bf16_bits(qh)
-            k[b, i] = to_bf16_bits(kh)
-            v[b, i] = to_bf16_bits(vh)
+
+    def one(job):
+        b, i, h = job
+        qh, kh, vh = head_qkv(w, b, h, coords)
+        q[b, i] = to_bf16_bits(qh)
+        k[b, i] = to_bf16_bits(kh)
+        v[b, i] = to_bf16_bits(vh)
+
+    jobs = [(b, i, h) for b in range(w.B) for i, h in enumerate(heads)]
+    n = threads or min(len(jobs), os.cpu_count() or 1, 16)
+    if n <= 1:
+        for job in jobs:
+            one(job)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(n) as ex:
+            list(ex.map(one, jobs))
     return q, k, v
 
 

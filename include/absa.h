@@ -1,0 +1,169 @@
+/*
+ * absa.h -- C ABI of the B200 (sm_100a) AB-Attention hot path:
+ * IBCS block selector, SIP sampler and Horvitz-Thompson sparse attention
+ * over 4-token key/value blocks, plus a dense attention kernel for
+ * comparison.
+ *
+ * Method source: "AB-Attention speeds up video generation by up to 2.23x and
+ * skips 92% of attention" (news.hamidun.com), section "AB-Attention's three
+ * techniques" -- IBCS paragraph (selector), SIP paragraph (sampler and 1/pi
+ * logit shift), third paragraph (4-token blocks gathered into full tensor-core
+ * tiles, plan reused for four denoising steps); and the HF daily-papers
+ * summary (zerohour.day) "Key facts": no token permutation, sub-tile blocks
+ * packed into full tensor-core tiles.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are caller-owned DEVICE memory; q, k, v, o are bf16 [B,H,N,d]
+ *    row-major (d fastest).  Token n of a T x Hg x Wg latent grid is
+ *    n = (t*Hg + y)*Wg + x and is never permuted.
+ *  - Query block qb holds tokens 128*qb .. min(128*qb+127, N-1)
+ *    (NQB = ceil(N/128)); key/value block j holds tokens 4j .. min(4j+3, N-1)
+ *    (NKB = ceil(N/4)).
+ *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  The
+ *    library never allocates, frees or synchronises, except absa_plan_check,
+ *    which synchronises the stream to read the device status word.
+ *  - Pointers must be 16-byte aligned.  Host-detectable errors return before
+ *    any launch; launch failures return ABSA_ERR_CUDA; errors seen on the
+ *    device are OR-ed into a device status word (ABSA_DEVFLAG_*).
+ *  - No CPU fallback: unsupported shapes return ABSA_ERR_UNSUPPORTED.
+ *  - Inputs are never written.
+ */
+#ifndef ABSA_H
+#define ABSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ABSA_OK = 0,
+    ABSA_ERR_INVALID_ARG = 1,   /* bad pointer, alignment, size or field        */
+    ABSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (d, block sizes)   */
+    ABSA_ERR_WORKSPACE = 3,     /* workspace smaller than absa_workspace_bytes  */
+    ABSA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed         */
+    ABSA_ERR_PLAN_OVERFLOW = 5, /* a sample exceeded the plan capacity          */
+    ABSA_ERR_BAD_PLAN = 6,      /* plan count/index out of range (seen on GPU)  */
+    ABSA_ERR_TIMEOUT = 7        /* a bounded device wait ran out                */
+} absa_status;
+
+/* Bits of the device status word (plan->status / the status argument). */
+#define ABSA_DEVFLAG_OVERFLOW 1
+#define ABSA_DEVFLAG_BAD_PLAN 2
+#define ABSA_DEVFLAG_TIMEOUT 4
+
+typedef struct {
+    int32_t B, H, N, d;     /* batch, heads, tokens (= T*Hg*Wg), head dim (64|128)   */
+    int32_t T, Hg, Wg;      /* latent grid; token n = (t*Hg + y)*Wg + x               */
+    int32_t q_block;        /* must be 128 (IBCS paragraph: blocks of 128 queries)    */
+    int32_t kv_block;       /* must be 4 (third paragraph: 4-token KV blocks)         */
+    int32_t n_clusters;     /* must be 8 (IBCS paragraph: 8 clusters per block)       */
+    int32_t kmeans_iters;   /* Lloyd rounds, 1..16 (3 in every workload)              */
+    int32_t budget_blocks;  /* n: expected KV blocks per query block; n >= NKB = dense */
+    uint64_t seed;          /* SIP draw seed                                          */
+    float softmax_scale;    /* logit scale, normally 1/sqrt(d)                        */
+} absa_params;
+
+typedef struct {
+    /* All arrays are caller-owned device memory sized from absa_plan_capacity. */
+    int32_t n_qblocks;      /* NQB                                                   */
+    int32_t n_kvblocks;     /* NKB                                                   */
+    int32_t capacity;       /* entries per row (>= absa_plan_capacity)               */
+    int32_t *counts;        /* [B,H,NQB] taken blocks per row (clipped to capacity)  */
+    int32_t *kv_index;      /* [B,H,NQB,capacity] ascending block ids, valid to count */
+    float *log_pi;          /* [B,H,NQB,capacity] ln(pi) of each entry (0 if pi = 1)  */
+    uint64_t *r_R;          /* [B,H,NQB,2] audit: r*, R* of the integer pi solve      */
+    int32_t *status;        /* one device word, OR of ABSA_DEVFLAG_*                  */
+} absa_plan;
+
+/* Library version string. */
+const char *absa_version(void);
+
+/* Human-readable name of a status code (static storage). */
+const char *absa_status_string(absa_status s);
+
+/* Validate a parameter block (host only).  Returns ABSA_OK, INVALID_ARG or
+ * UNSUPPORTED. */
+absa_status absa_check_params(const absa_params *p);
+
+/* Plan row capacity for p: min(NKB, roundup32(n + ceil(8*sqrt(n)) + 32)),
+ * i.e. the budget plus eight standard deviations of a Poisson sample size
+ * (SIP paragraph: blocks are drawn, so the sample size varies).  Returns -1
+ * if p is invalid. */
+int32_t absa_plan_capacity(const absa_params *p);
+
+/* Bytes of workspace absa_select_scores / absa_select_plan need.  Layout,
+ * each region starting at a 256-byte boundary in this order:
+ *   kbar_hi  bf16 [B,H,NKB,d]   mean key of every 4-token block, high part
+ *   kbar_lo  bf16 [B,H,NKB,d]   low part (kbar ~= hi + lo to 2^-17)
+ *   mu       f32  [B,H,NQB,8,d] final k-means centroids
+ *   mu_hi    bf16 [B,H,NQB,8,d] split of mu for the tensor-core score
+ *   mu_lo    bf16 [B,H,NQB,8,d]
+ *   w        f32  [B,H,NQB,8]   centroid weights |c| / n_valid
+ *   assign   u8   [B,H,NQB,128] final assignment (255 for padded rows)
+ * The regions after kbar_lo are readable audit outputs of the last call.
+ * Returns 0 if p is invalid. */
+size_t absa_workspace_bytes(const absa_params *p);
+
+/* IBCS selector (IBCS paragraph): for every (b,h) pool the keys of each
+ * 4-token block into their mean, run the per-128-query-block k-means
+ * (8 clusters, kmeans_iters Lloyd rounds in fp32, initial centroids the
+ * queries at offsets floor(c*m/8), ties to the lowest index, empty clusters
+ * keep their centroid), weight each centroid by its share of the block's m
+ * valid queries, and write
+ *   scores[b,h,qb,j] = sum_c w_c * softmax_j(softmax_scale * mu_c . kbar_j)
+ * (f32 [B,H,NQB,NKB], each row sums to 1).  ws must hold
+ * absa_workspace_bytes(p) bytes (ABSA_ERR_WORKSPACE otherwise). */
+absa_status absa_select_scores(const absa_params *p, const void *q, const void *k,
+                               float *scores, void *ws, size_t ws_bytes, void *stream);
+
+/* SIP sampler (SIP paragraph) on a score array [B,H,NQB,NKB] f32.
+ * Integer inclusion probabilities: q_j = max(1, floor(s_j * 2^32)) (NaN or
+ * negative -> 1, at most 2^32); from C = {} repeat r = n - |C|,
+ * R = sum_{j not in C} q_j, C += {j : r*q_j >= R} until C is unchanged;
+ * pi_j = 1 on C, r*q_j/R elsewhere, so sum pi = n exactly.  Poisson draws:
+ * u_j = mix(mix(row*NKB + j + 0x9E3779B97F4A7C15) ^ seed) >> 32 with mix the
+ * SplitMix64 output function and row = (b*H + h)*NQB + qb; block j is taken
+ * iff j in C or u_j * R < r*q_j * 2^32.  Taken blocks are written ascending
+ * with log_pi = 0 (capped) or (float)ln((double)(r*q_j)/R).  n >= NKB takes
+ * every block.  Resets plan->status first; a row with more than
+ * plan->capacity blocks keeps the first `capacity` and sets
+ * ABSA_DEVFLAG_OVERFLOW.  Requires NKB <= 49152. */
+absa_status absa_sample_plan(const absa_params *p, const float *scores, const absa_plan *plan,
+                             void *stream);
+
+/* absa_select_scores followed by absa_sample_plan (one plan per call; the
+ * third paragraph's schedule recomputes it every fourth denoising step and
+ * reuses it in between). */
+absa_status absa_select_plan(const absa_params *p, const void *q, const void *k, float *scores,
+                             const absa_plan *plan, void *ws, size_t ws_bytes, void *stream);
+
+/* Horvitz-Thompson sparse attention (SIP paragraph; third paragraph): for
+ * every valid query i of block qb, over the tokens t of the plan's blocks in
+ * ascending order, l_t = softmax_scale * q_i . k_t - log_pi(block of t) and
+ * o_i = sum_t softmax(l)_t v_t; an empty plan row gives o_i = 0.  The
+ * selected 4-token blocks are gathered by index into 128-token tensor-core
+ * tiles (tcgen05, bf16 operands, f32 accumulation); tokens are not
+ * permuted.  The plan may come from an earlier step (plan reuse).  Plan
+ * counts above capacity or indices outside [0, NKB) are rejected on the
+ * device (ABSA_DEVFLAG_BAD_PLAN, the row is written as zeros). */
+absa_status absa_sparse_attention(const absa_params *p, const void *q, const void *k,
+                                  const void *v, const absa_plan *plan, void *o, void *stream);
+
+/* Dense softmax attention (the full-attention reference of the pages'
+ * evaluation) with the same tile machinery over contiguous keys.  status is
+ * a device word for ABSA_DEVFLAG_TIMEOUT (may be NULL). */
+absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,
+                                 const void *v, void *o, int32_t *status, void *stream);
+
+/* Synchronise `stream`, read plan->status and map it to a status code
+ * (TIMEOUT > BAD_PLAN > OVERFLOW > OK).  Does not clear the word. */
+absa_status absa_plan_check(const absa_plan *plan, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ABSA_H */
