@@ -35,20 +35,28 @@ L2_FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only this many heads (profiling captures); 0 = all 40")
+    ap.add_argument("--dense-reps", type=int, default=3)
     return ap.parse_args()
 
 
-def workload():
+def workload(heads=0):
     from block_sparse_attention_selector_b200 import synthetic
 
-    return synthetic.WAN480
+    w = synthetic.WAN480
+    if heads:
+        import dataclasses
+
+        w = dataclasses.replace(w, H=int(heads), name=f"{w.name}_{int(heads)}heads")
+    return w
 
 
 def config_of(w, extra=None):
@@ -145,7 +153,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -226,7 +234,7 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    w = workload()
+    w = workload(args.heads)
     q_bits, k_bits, v_bits = synthetic.layer_qkv_bits(w)
 
     def to_dev(b):
@@ -254,6 +262,7 @@ def run_ours(args):
         if ev is not None:
             ev[3].record(stream)
 
+    clocks = ClockSampler(dev.index).__enter__()  # sampling starts before the warm-up
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         step()
@@ -266,11 +275,11 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
-        for i in range(K):
-            flush.zero_()
-            step(events[i])
-        torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
     if world > 1:
         dist.barrier()
     plan.check()
@@ -294,7 +303,7 @@ def run_ours(args):
     # dense reference kernel on the same shapes (companion number)
     ev_d = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     dense_ms = []
-    for _ in range(3):
+    for _ in range(args.dense_reps):
         flush.zero_()
         ev_d[0].record(stream)
         absa.dense_reference(p, q, k, v, o)
@@ -307,7 +316,7 @@ def run_ours(args):
                      for b in (q_bits, k_bits, v_bits))
     o_h = torch.empty_like(q_h).pin_memory()
     e2e = []
-    for i in range(1 + args.e2e_steps):
+    for i in range(1 + args.e2e_steps if args.e2e_steps > 0 else 0):
         flush.zero_()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -325,7 +334,7 @@ def run_ours(args):
     te = torch.tensor([float(np.sum(e2e))], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / (len(e2e) * world)
+    e2e_ms = float(te.item()) / (max(1, len(e2e)) * world) if e2e else None
 
     peak_tf, hbm_gbs, peak_src = measured_peaks()
     att_ms = float(att.mean())
@@ -344,8 +353,9 @@ def run_ours(args):
                 "breakdown_ms": {"select_scores": float(sel.mean()), "sample": float(smp.mean()),
                                  "sparse_attention": att_ms},
                 "plan_reuse_ms_per_call": float(sel.mean() + smp.mean()) / 4 + att_ms,
-                "dense_reference_ms": float(np.median(dense_ms)),
-                "dense_tflops": 4.0 * w.d * w.N * w.N * w.B * w.H / (np.median(dense_ms) * 1e-3) / 1e12,
+                "dense_reference_ms": float(np.median(dense_ms)) if dense_ms else None,
+                "dense_tflops": (4.0 * w.d * w.N * w.N * w.B * w.H / (np.median(dense_ms) * 1e-3)
+                                 / 1e12) if dense_ms else None,
                 "mean_blocks_per_row": float(counts.mean()),
                 "selector_hbm_frac_of_measured": sel_bytes / (float(sel.mean()) * 1e-3) / 1e9 / hbm_gbs,
             }),

@@ -58,20 +58,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` nanoseconds pass, without spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity.  Returns false (after setting the
-// timeout flag in *status and *abort) if it does not complete in time or if
-// another thread of the CTA already gave up.
+// timeout flag in *status and *abort) if it does not complete within about
+// kWaitLimitCycles, or if another thread of the CTA already gave up.  The
+// clock and the abort flag are read once every 16 sleeps so that waiting
+// warps take almost no issue slots.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
                                           volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
-    long long t0 = clock64();
-    for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            *abort = 1;
-            if (status) atomicOr(status, ABSA_DEVFLAG_TIMEOUT);
-            return false;
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((i & 15u) == 0) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                *abort = 1;
+                if (status) atomicOr(status, ABSA_DEVFLAG_TIMEOUT);
+                return false;
+            }
         }
     }
 }
@@ -86,6 +105,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 }
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the pending count is raised now and lowered on completion, so the thread
+// also makes its own regular arrive).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {

@@ -31,7 +31,10 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
                           uint64_t *r_R, int32_t *status, cudaStream_t stream);
 
 // K5 (dense = false) / K6 (dense = true): attention over 128-token tiles.
-cudaError_t launch_attention(bool dense, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+// tq: q as [B*H*N, d] bf16 with a 64 x 128 box; tk / tv: k / v with a 64 x 4
+// box (sparse: one 4-token block per box) or a 64 x 128 box (dense tiles).
+cudaError_t launch_attention(bool dense, const CUtensorMap &tq, const CUtensorMap &tk,
+                             const CUtensorMap &tv, const __nv_bfloat16 *k,
                              const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N, int nqb,
                              int nkb, int d, float softmax_scale, const int32_t *counts,
                              const int32_t *kv_index, const float *log_pi, int cap,

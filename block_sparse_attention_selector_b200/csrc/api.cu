@@ -72,13 +72,14 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (cols fastest), box 64 x 128 with 128-byte swizzle.
-bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int cols) {
+// 2-D bf16 tensor [rows, cols] (cols fastest), box 64 x box_rows with 128-byte swizzle.
+bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int cols,
+                   int box_rows = 128) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estride[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), gdim, gstride,
               box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -133,7 +134,8 @@ absa_status absa_check_params(const absa_params *p) {
     if (p->d != 64 && p->d != 128) return ABSA_ERR_UNSUPPORTED;
     const Dims dm = dims_of(p);
     // TMA row coordinates and per-CTA indices are 32-bit
-    if (dm.BH * dm.nkb >= (int64_t)1 << 31 || dm.BH * dm.nqb * 8 >= (int64_t)1 << 31)
+    if (dm.BH * dm.nkb >= (int64_t)1 << 31 || dm.BH * dm.nqb * 8 >= (int64_t)1 << 31 ||
+        dm.BH * p->N + 128 >= (int64_t)1 << 31)
         return ABSA_ERR_UNSUPPORTED;
     if (dm.nkb > kSampleMaxKvBlocks) return ABSA_ERR_UNSUPPORTED;
     return ABSA_OK;
@@ -255,11 +257,17 @@ absa_status absa_sparse_attention(const absa_params *p, const void *q, const voi
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
         return ABSA_ERR_INVALID_ARG;
     const Dims dm = dims_of(p);
-    return from_cuda(launch_attention(
-        false, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), dm.BH, p->N,
-        dm.nqb, dm.nkb, p->d, p->softmax_scale, plan->counts, plan->kv_index, plan->log_pi,
-        plan->capacity, plan->status, reinterpret_cast<cudaStream_t>(stream)));
+    CUtensorMap tq, tk, tv;
+    // sparse gathers: one 4-row box (one 4-token block) per 64-column region
+    if (!make_map_bf16(&tq, q, dm.BH * p->N, p->d) || !make_map_bf16(&tk, k, dm.BH * p->N, p->d, 4) ||
+        !make_map_bf16(&tv, v, dm.BH * p->N, p->d, 4))
+        return ABSA_ERR_CUDA;
+    return from_cuda(launch_attention(false, tq, tk, tv, static_cast<const __nv_bfloat16 *>(k),
+                                      static_cast<const __nv_bfloat16 *>(v),
+                                      static_cast<__nv_bfloat16 *>(o), dm.BH,
+                                      p->N, dm.nqb, dm.nkb, p->d, p->softmax_scale, plan->counts,
+                                      plan->kv_index, plan->log_pi, plan->capacity, plan->status,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,
@@ -271,11 +279,16 @@ absa_status absa_dense_reference(const absa_params *p, const void *q, const void
         return ABSA_ERR_INVALID_ARG;
     if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return ABSA_ERR_INVALID_ARG;
     const Dims dm = dims_of(p);
-    return from_cuda(launch_attention(
-        true, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), dm.BH, p->N,
-        dm.nqb, dm.nkb, p->d, p->softmax_scale, nullptr, nullptr, nullptr, 0, status,
-        reinterpret_cast<cudaStream_t>(stream)));
+    CUtensorMap tq, tk, tv;
+    if (!make_map_bf16(&tq, q, dm.BH * p->N, p->d) || !make_map_bf16(&tk, k, dm.BH * p->N, p->d) ||
+        !make_map_bf16(&tv, v, dm.BH * p->N, p->d))
+        return ABSA_ERR_CUDA;
+    return from_cuda(launch_attention(true, tq, tk, tv, static_cast<const __nv_bfloat16 *>(k),
+                                      static_cast<const __nv_bfloat16 *>(v),
+                                      static_cast<__nv_bfloat16 *>(o), dm.BH,
+                                      p->N, dm.nqb, dm.nkb, p->d, p->softmax_scale, nullptr,
+                                      nullptr, nullptr, 0, status,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 absa_status absa_plan_check(const absa_plan *plan, void *stream) {

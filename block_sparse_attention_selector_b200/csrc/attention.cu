@@ -6,12 +6,16 @@
 // -ln(pi) (SIP paragraph); the 4-token blocks are gathered by index into
 // full-size tensor-core tiles, tokens are not permuted (third paragraph).
 //
-// Kernel design (one CTA per (b, h, 128-query block), 256 threads):
-//   warps 0-3  softmax: thread t owns query row t = TMEM lane t
-//   warps 4-6  loaders: cp.async gathers of 32 blocks (= 128 key rows) per
-//              tile into SW128 shared-memory tiles, K and V in separate
-//              2-stage rings, plus the tile's per-column logit bias
-//   warp 7     TMEM owner and MMA issuer (one thread):
+// Kernel design (one CTA per (b, h, 128-query block), 512 threads):
+//   warps 0-7   softmax, two warpgroups: warpgroup g handles columns
+//               64g..64g+63 of each S tile for all 128 rows (thread = TMEM
+//               lane = query row); the row max is exchanged through shared
+//               memory; warpgroup g rescales and stores output columns
+//               (d/2)g .. (d/2)g + d/2 - 1
+//   warps 8-14  loaders: TMA gathers of 32 blocks (= 128 key rows) per tile
+//               into SW128 shared-memory tiles, K and V in separate 2-stage
+//               rings, plus the tile's per-column logit bias
+//   warp 15     TMEM owner and MMA issuer (one thread):
 //              S_j = Q K_j^T  -> TMEM (two 128-column buffers)
 //              O  += P_j V_j  -> TMEM (D columns), P_j bf16 in shared memory
 // Softmax works in the exp2 domain: x = log2(e) * scale * (q.k) + bias with
@@ -33,27 +37,40 @@ struct AttnSmem {
     static constexpr int kVOff = kKOff + 2 * kKVBytes;         // [2] stages
     static constexpr int kPOff = kVOff + 2 * kKVBytes;         // 128 x 128 bf16
     static constexpr int kBiasOff = kPOff + 2 * kTile;         // [2][128] f32
-    static constexpr int kBarOff = kBiasOff + 2 * 128 * 4;
-    static constexpr int kBytes = kBarOff + 18 * 8 + 2 * 32 * 4;
+    static constexpr int kRedOff = kBiasOff + 2 * 128 * 4;    // [2][2][128] f32 exchange
+    static constexpr int kBarOff = kRedOff + 4 * 128 * 4;
+    static constexpr int kBytes = kBarOff + 24 * 8;
     // keep one CTA per SM so that the 512-column TMEM allocation never waits
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
 };
 
-constexpr int kLoadWarps = 3;
-constexpr int kLoadThreads = 32 * kLoadWarps;
-constexpr int kMmaWarp = 4 + kLoadWarps;
-constexpr int kAttnThreads = 32 * (kMmaWarp + 1);  // 256
+constexpr int kSoftmaxWarps = 8;              // two warpgroups, 64 columns each
+constexpr int kLoadWarp = kSoftmaxWarps;      // first loader warp
+constexpr int kLoadWarps = 7;                 // warps issuing TMA boxes
+constexpr int kMmaWarp = kLoadWarp + kLoadWarps;   // 15
+constexpr int kAttnThreads = 32 * (kMmaWarp + 1);  // 512
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Loaders.  Sparse mode: a tile's 32 blocks x (d/64) column regions are 4-row
+// TMA boxes (512 bytes each) placed at rows 4i..4i+3 of the SW128 tile; the
+// box swizzle follows the shared-memory address, so a box in the upper half
+// of a 1024-byte atom lands in that half's chunk order.  The boxes are spread
+// over 7 warps (box p goes to warp p % 7): a single warp sustains only about
+// 9 bytes/clock of such small boxes, several warps several times that.  Block
+// ids and log(pi) of the next tile are prefetched while the current tile is
+// issued.  Dense mode: one 128-row box per region from one lane.
+// K and V use separate 2-stage rings; the logit bias of the tile travels with
+// V (every loader warp arrives on v_full after writing its columns).
 template <int D, bool DENSE>
 __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
-    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-    const __nv_bfloat16 *__restrict__ v, __nv_bfloat16 *__restrict__ o, int N, int nqb, int nkb,
-    float scale_log2, const int32_t *__restrict__ counts, const int32_t *__restrict__ kv_index,
-    const float *__restrict__ log_pi, int cap, int32_t *status) {
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ k,
+    const __nv_bfloat16 *__restrict__ v, __nv_bfloat16 *__restrict__ o, int N, int nqb,
+    int nkb, float scale_log2, const int32_t *__restrict__ counts,
+    const int32_t *__restrict__ kv_index, const float *__restrict__ log_pi, int cap,
+    int32_t *status) {
     using S = AttnSmem<D>;
-    constexpr int CH = D / 8;  // 16-byte chunks per row
     extern __shared__ uint8_t attn_smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -70,7 +87,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     uint64_t *p_free = bars + 14;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 16);
-    int *blk_s = reinterpret_cast<int *>(bars + 18);  // [2][32] block ids of the tile
+    float *red = reinterpret_cast<float *>(sm + S::kRedOff);  // [parity][half][row]
+    uint64_t *xchg = bars + 17;     // [2] row-max exchange of the two softmax warpgroups
+    uint64_t *xchg_end = bars + 19; // row-sum exchange before the epilogue
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -80,21 +99,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     const int m = min(128, N - qb * 128);
 
     if (tid == 0) {
-        mbar_init(q_full, kLoadThreads);
+        mbar_init(q_full, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(k_full + s, kLoadThreads);
+            mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
-            mbar_init(v_full + s, kLoadThreads);
+            mbar_init(v_full + s, DENSE ? 1 : kLoadWarps);
             mbar_init(v_empty + s, 1);
             mbar_init(s_full + s, 1);
-            mbar_init(s_free + s, 4);
+            mbar_init(s_free + s, kSoftmaxWarps);
         }
-        mbar_init(p_full, 4);
+        mbar_init(p_full, kSoftmaxWarps);
         mbar_init(p_free, 1);
+        mbar_init(xchg, kSoftmaxWarps);
+        mbar_init(xchg + 1, kSoftmaxWarps);
+        mbar_init(xchg_end, kSoftmaxWarps);
         *abort_flag = 0;
         mbar_fence_init();
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
+    // Rows of a partial tile that no box overwrites must hold finite values
+    // (P = 0 there, and 0 * NaN would poison O): clear the K/V rings once.
+    for (int i = tid; i < 4 * S::kKVBytes / 16; i += kAttnThreads)
+        reinterpret_cast<uint4 *>(sm + S::kKOff)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
 
     // number of plan entries; reject a malformed plan row (it is written as zeros)
     int count;
@@ -121,133 +148,193 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     const uint32_t tmem = *tmem_slot;
     const uint32_t tmem_o = tmem + 256;
 
-    if (warp >= 4 && warp < 4 + kLoadWarps) {
+    if (warp >= kLoadWarp && warp < kLoadWarp + kLoadWarps) {
         // ------------------------------------------------------------ loaders
-        const int lt = tid - 128;
-        const uint32_t q_s = smem_u32(sm + S::kQOff);
-        const __nv_bfloat16 *qsrc = q + (bh * N + (int64_t)qb * 128) * D;
-        for (int idx = lt; idx < 128 * CH; idx += kLoadThreads) {
-            const int r = idx / CH, c = idx % CH;
-            const bool ok = r < m;
-            cp_async16(q_s + (c >> 3) * S::kTile + sw128_offset(r, c & 7),
-                       qsrc + (int64_t)(ok ? r : 0) * D + c * 8, ok ? 16u : 0u);
+        const int lw = warp - kLoadWarp;      // 0..6
+        const int64_t row0 = bh * N;          // first token row of this head
+        if (lw == 0 && lane == 0 && T > 0) {
+            mbar_arrive_expect_tx(q_full, S::kQBytes);
+            const uint32_t q_s = smem_u32(sm + S::kQOff);
+            for (int r = 0; r < S::kRegions; ++r)
+                tma_load_2d(q_s + r * S::kTile, &tm_q, 64 * r, (int)(row0 + qb * 128), q_full);
         }
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(q_full);
-
-        const __nv_bfloat16 *kh = k + bh * (int64_t)N * D;
-        const __nv_bfloat16 *vh = v + bh * (int64_t)N * D;
         const int32_t *idx_row = DENSE ? nullptr : kv_index + row * cap;
         const float *lp_row = DENSE ? nullptr : log_pi + row * cap;
+        // box p = lw + 7 * lane of a tile: block slot p / R, region p % R
+        constexpr int R = S::kRegions;
+        const int pbox = lw + kLoadWarps * lane;
+        const int slot = pbox / R, reg = pbox % R;
+        const bool has_box = pbox < 32 * R;
+        // prefetch of block id and log(pi) for tile 0
+        int b_next = -1;
+        float lp_next = 0.f;
+        if (!DENSE && has_box && slot < count) {
+            b_next = __ldg(idx_row + slot);
+            lp_next = __ldg(lp_row + slot);
+        }
         bool ok = true;
         for (int j = 0; j < T && ok; ++j) {
             const int st = j & 1;
             const int nb = min(32, count - 32 * j);
-            int *blk_ids = blk_s + st * 32;
-            if (lt < 32) blk_ids[lt] = lt < nb ? (DENSE ? 32 * j + lt : __ldg(idx_row + 32 * j + lt)) : -1;
-            asm volatile("bar.sync 2, %0;" ::"n"(kLoadThreads) : "memory");
-            if (j >= 2 && !mbar_wait(k_empty + st, ((j - 2) >> 1) & 1, status, abort_flag)) {
-                ok = false;
-                break;
+            const int b = b_next;
+            const float lpv = lp_next;
+            if (!DENSE) {  // prefetch the next tile's entries
+                b_next = -1;
+                const int e = 32 * (j + 1) + slot;
+                if (has_box && e < count) {
+                    b_next = __ldg(idx_row + e);
+                    lp_next = __ldg(lp_row + e);
+                }
+            }
+            if (j >= 2) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(k_empty + st, ((j - 2) >> 1) & 1, status, abort_flag));
+                if (!ok) break;
             }
             const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
-            for (int idx = lt; idx < 128 * CH; idx += kLoadThreads) {
-                const int r = idx / CH, c = idx % CH;
-                const int b = blk_ids[r >> 2];
-                const int t = 4 * b + (r & 3);
-                const bool valid = b >= 0 && t < N;
-                cp_async16(k_s + (c >> 3) * S::kTile + sw128_offset(r, c & 7),
-                           kh + (int64_t)(valid ? t : 0) * D + c * 8, valid ? 16u : 0u);
+            if (DENSE) {
+                if (lw == 0 && lane == 0) {
+                    mbar_arrive_expect_tx(k_full + st, S::kKVBytes);
+                    for (int r = 0; r < R; ++r)
+                        tma_load_2d(k_s + r * S::kTile, &tm_k, 64 * r, (int)(row0 + 128 * j),
+                                    k_full + st);
+                }
+            } else {
+                if (lw == 0 && lane == 0) mbar_arrive_expect_tx(k_full + st, nb * 512 * R);
+                if (b >= 0)
+                    tma_load_2d(k_s + reg * S::kTile + slot * 512, &tm_k, 64 * reg,
+                                (int)(row0 + 4 * b), k_full + st);
             }
-            cp_async_commit();
-            if (j >= 1) {  // V of the previous tile has landed: publish it
-                cp_async_wait<1>();
-                fence_proxy_async_smem();
-                mbar_arrive(v_full + ((j - 1) & 1));
-            }
-            if (j >= 2 && !mbar_wait(v_empty + st, ((j - 2) >> 1) & 1, status, abort_flag)) {
-                ok = false;
-                break;
+            if (j >= 2) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(v_empty + st, ((j - 2) >> 1) & 1, status, abort_flag));
+                if (!ok) break;
             }
             const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
-            for (int idx = lt; idx < 128 * CH; idx += kLoadThreads) {
-                const int r = idx / CH, c = idx % CH;
-                const int b = blk_ids[r >> 2];
-                const int t = 4 * b + (r & 3);
-                const bool valid = b >= 0 && t < N;
-                cp_async16(v_s + (c >> 3) * S::kTile + sw128_offset(r, c & 7),
-                           vh + (int64_t)(valid ? t : 0) * D + c * 8, valid ? 16u : 0u);
+            if (DENSE) {
+                if (lw == 0) {
+                    float4 bias;
+                    const int t0 = 128 * j + 4 * lane;
+                    bias.x = t0 < N ? 0.f : -INFINITY;
+                    bias.y = t0 + 1 < N ? 0.f : -INFINITY;
+                    bias.z = t0 + 2 < N ? 0.f : -INFINITY;
+                    bias.w = t0 + 3 < N ? 0.f : -INFINITY;
+                    reinterpret_cast<float4 *>(bias_s + st * 128)[lane] = bias;
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
+                        for (int r = 0; r < R; ++r)
+                            tma_load_2d(v_s + r * S::kTile, &tm_v, 64 * r, (int)(row0 + 128 * j),
+                                        v_full + st);
+                    }
+                }
+            } else {
+                if (has_box && reg == 0) {  // logit bias of the block's 4 columns
+                    float4 bias = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                    if (b >= 0) {
+                        const float sh = -lpv * kLog2e;
+                        const int t0 = 4 * b;
+                        bias.x = t0 < N ? sh : -INFINITY;
+                        bias.y = t0 + 1 < N ? sh : -INFINITY;
+                        bias.z = t0 + 2 < N ? sh : -INFINITY;
+                        bias.w = t0 + 3 < N ? sh : -INFINITY;
+                    }
+                    reinterpret_cast<float4 *>(bias_s + st * 128)[slot] = bias;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    if (lw == 0)
+                        mbar_arrive_expect_tx(v_full + st, nb * 512 * R);
+                    else
+                        mbar_arrive(v_full + st);
+                }
+                if (b >= 0)
+                    tma_load_2d(v_s + reg * S::kTile + slot * 512, &tm_v, 64 * reg,
+                                (int)(row0 + 4 * b), v_full + st);
             }
-            for (int col = lt; col < 128; col += kLoadThreads) {  // logit bias per column
-                const int b = blk_ids[col >> 2];
-                float bias = -INFINITY;
-                if (b >= 0 && 4 * b + (col & 3) < N)
-                    bias = DENSE ? 0.f : -__ldg(lp_row + 32 * j + (col >> 2)) * kLog2e;
-                bias_s[st * 128 + col] = bias;
-            }
-            cp_async_commit();
-            cp_async_wait<1>();  // K of this tile has landed
-            fence_proxy_async_smem();
-            mbar_arrive(k_full + st);
         }
-        if (ok && T > 0) {
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            mbar_arrive(v_full + ((T - 1) & 1));
-        }
-        cp_async_wait<0>();
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // Issues S_j = Q K_j^T as soon as K_j has landed and S buffer j%2 is
+        // free, and O += P_j V_j as soon as P_j is written; whichever is ready
+        // first goes first, so neither waits behind the other's operands.
+        if (lane == 0 && T > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
             const uint32_t q_s = smem_u32(sm + S::kQOff);
             const uint32_t p_s = smem_u32(sm + S::kPOff);
-            bool ok = T == 0 || mbar_wait(q_full, 0, status, abort_flag);
-            auto issue_pv = [&](int jj) -> bool {
-                const int st = jj & 1;
-                if (!mbar_wait(v_full + st, (jj >> 1) & 1, status, abort_flag)) return false;
-                if (!mbar_wait(p_full, jj & 1, status, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
+            bool ok = mbar_wait(q_full, 0, status, abort_flag);
+            int js = 0, jp = 0;  // next S tile, next PV tile
+            long long t0 = clock64();
+            uint32_t spins = 0;
+            while (ok && jp < T) {
+                bool progressed = false;
+                if (js < T && js < jp + 2) {
+                    const int st = js & 1;
+                    if (mbar_try_wait(k_full + st, (js >> 1) & 1) &&
+                        (js < 2 || mbar_try_wait(s_free + st, ((js - 2) >> 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = sw128_desc(p_s + (ks >> 2) * S::kTile + (ks & 3) * 32, 16, 1024);
-                    const uint64_t b = sw128_desc(v_s + ks * 2048, S::kTile, 1024);
-                    tc_mma_f16(tmem_o, a, b, idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
+                            tc_mma_f16(tmem + st * 128, sw128_desc(q_s + off, 16, 1024),
+                                       sw128_desc(k_s + off, 16, 1024), idesc_s,
+                                       ks > 0 ? 1u : 0u);
+                        }
+                        tc_commit(s_full + st);
+                        tc_commit(k_empty + st);
+                        ++js;
+                        progressed = true;
+                    }
                 }
-                tc_commit(p_free);
-                tc_commit(v_empty + st);
-                return true;
-            };
-            for (int j = 0; ok && j < T; ++j) {
-                const int st = j & 1, b = j & 1;
-                if (!mbar_wait(k_full + st, (j >> 1) & 1, status, abort_flag)) break;
-                if (j >= 2 && !mbar_wait(s_free + b, ((j - 2) >> 1) & 1, status, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
+                if (jp < js) {
+                    const int st = jp & 1;
+                    if (mbar_try_wait(p_full, jp & 1) && mbar_try_wait(v_full + st, (jp >> 1) & 1)) {
+                        tc_fence_after();
+                        const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
-                    tc_mma_f16(tmem + b * 128, sw128_desc(q_s + off, 16, 1024),
-                               sw128_desc(k_s + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint64_t a =
+                                sw128_desc(p_s + (ks >> 2) * S::kTile + (ks & 3) * 32, 16, 1024);
+                            const uint64_t bdesc = sw128_desc(v_s + ks * 2048, S::kTile, 1024);
+                            tc_mma_f16(tmem_o, a, bdesc, idesc_o, (jp > 0 || ks > 0) ? 1u : 0u);
+                        }
+                        tc_commit(p_free);
+                        tc_commit(v_empty + st);
+                        ++jp;
+                        progressed = true;
+                    }
                 }
-                tc_commit(s_full + b);
-                tc_commit(k_empty + st);
-                if (j >= 1 && !issue_pv(j - 1)) {
-                    ok = false;
-                    break;
+                if (progressed) {
+                    spins = 0;
+                } else {
+                    __nanosleep(32);  // leave the issue slots to the softmax warps
+                    if ((++spins & 255u) == 0) {
+                        if (*abort_flag) {
+                            ok = false;
+                        } else if (spins == 256u) {
+                            t0 = clock64();  // start of this stall
+                        } else if (clock64() - t0 > kWaitLimitCycles) {
+                            *abort_flag = 1;
+                            if (status) atomicOr(status, ABSA_DEVFLAG_TIMEOUT);
+                            ok = false;
+                        }
+                    }
                 }
             }
-            if (ok && T > 0) issue_pv(T - 1);
         }
     } else {
         // ------------------------------------------------------------- softmax
-        const int r = tid;  // query row = TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t p_s = smem_u32(sm + S::kPOff);
+        // warpgroup `half` handles columns 64*half .. 64*half+63 of every S
+        // tile and output columns (D/2)*half ..; thread = TMEM lane = row.
+        const int half = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;  // query row = TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t p_s = smem_u32(sm + S::kPOff) + half * S::kTile;
+        const int cb = 64 * half;
+        constexpr int OC = D / 2;              // output columns of this half
+        const uint32_t o_cols = tmem_o + half * OC;
         float m_ref = -INFINITY, lsum = 0.f;
         bool ok = true;
         for (int j = 0; j < T; ++j) {
@@ -255,19 +342,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             ok = __all_sync(0xffffffffu, mbar_wait(s_full + b, (j >> 1) & 1, status, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[4][32];
+            uint32_t sv[2][32];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + b * 128 + ch * 32, sv[ch]);
+            for (int ch = 0; ch < 2; ++ch)
+                tmem_ld32(tmem + lane_base + b * 128 + cb + ch * 32, sv[ch]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free + b);
             ok = __all_sync(0xffffffffu, mbar_wait(v_full + b, (j >> 1) & 1, status, abort_flag));
             if (!ok) break;
-            const float *bias = bias_s + b * 128;
-            float tmax = -INFINITY;
+            const float *bias = bias_s + b * 128 + cb;
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
+            for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
                     const float4 bb = *reinterpret_cast<const float4 *>(bias + ch * 32 + i);
@@ -279,8 +367,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                     sv[ch][i + 1] = __float_as_uint(x1);
                     sv[ch][i + 2] = __float_as_uint(x2);
                     sv[ch][i + 3] = __float_as_uint(x3);
-                    tmax = fmaxf(tmax, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+                    const int a = (i >> 2) & 3;
+                    mx4[a] = fmaxf(mx4[a], fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
                 }
+            // row max over both halves: exchange through shared memory
+            float *rx = red + (j & 1) * 256;
+            rx[half * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xchg + (j & 1));
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(xchg + (j & 1), (j >> 1) & 1, status, abort_flag));
+            if (!ok) break;
+            const float tmax = fmaxf(rx[r], rx[128 + r]);
             if (j == 0) m_ref = tmax;
             const bool need = j > 0 && tmax > m_ref + kRescaleThreshold;
             const bool any_need = __any_sync(0xffffffffu, need);
@@ -292,58 +390,67 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 if (!ok) break;
             }
             const float moff = -m_ref;
-            float acc = 0.f;
+            float acc8[8];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int i = 0; i < 8; ++i) acc8[i] = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {  // 8 columns = one 16-byte chunk
                     float p[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         p[e] = ex2(__uint_as_float(sv[ch][g * 8 + e]) + moff);
-                        acc += p[e];
+                        acc8[e] += p[e];
                     }
-                    const int col = ch * 32 + g * 8;
-                    const uint32_t dst = p_s + (col >> 6) * S::kTile + sw128_offset(r, (col >> 3) & 7);
+                    const uint32_t dst = p_s + sw128_offset(r, ch * 4 + g);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
                                  "r"(pack_bf16x2(p[0], p[1])), "r"(pack_bf16x2(p[2], p[3])),
                                  "r"(pack_bf16x2(p[4], p[5])), "r"(pack_bf16x2(p[6], p[7]))
                                  : "memory");
                 }
             }
-            if (any_need) {  // lazy rescale of the running output by exp2(m_old - m_new)
+            if (any_need) {  // lazy rescale of this half's output columns
                 tc_fence_after();
                 lsum *= alpha;
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < OC / 32; ++ch) {
                     uint32_t ov[32];
-                    tmem_ld32(tmem_o + lane_base + ch * 32, ov);
+                    tmem_ld32(o_cols + lane_base + ch * 32, ov);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(tmem_o + lane_base + ch * 32, ov);
+                    tmem_st32(o_cols + lane_base + ch * 32, ov);
                 }
                 tmem_wait_st();
             }
-            lsum += acc;
+            lsum += ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
+                    ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        // epilogue: O / lsum -> bf16, valid rows only
-        __nv_bfloat16 *orow = o + (bh * N + (int64_t)qb * 128 + r) * D;
+        // epilogue: O / (sum over both halves) -> bf16, valid rows only
+        // (the parity buffer of tile T is free: its last readers passed tile T-1)
+        float *rs = red + (T & 1) * 256;
+        rs[half * 128 + r] = lsum;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xchg_end);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(xchg_end, 0, status, abort_flag));
+        const float ltot = rs[r] + rs[128 + r];
+        __nv_bfloat16 *orow = o + (bh * N + (int64_t)qb * 128 + r) * D + half * OC;
         if (T > 0 && ok) {
             ok = __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, status, abort_flag));
         }
         if (T > 0 && ok) {
             tc_fence_after();
-            const float inv = 1.f / lsum;
+            const float inv = 1.f / ltot;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+            for (int ch = 0; ch < OC / 32; ++ch) {
                 uint32_t ov[32];
-                tmem_ld32(tmem_o + lane_base + ch * 32, ov);
+                tmem_ld32(o_cols + lane_base + ch * 32, ov);
                 tmem_wait_ld();
                 if (r < m) {
 #pragma unroll
@@ -364,7 +471,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         } else if (T == 0 && r < m) {
             const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int c = 0; c < CH; ++c) *reinterpret_cast<uint4 *>(orow + c * 8) = z;
+            for (int c = 0; c < OC / 8; ++c) *reinterpret_cast<uint4 *>(orow + c * 8) = z;
         }
     }
     tc_fence_before();
@@ -377,7 +484,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
 }
 
 template <int D, bool DENSE>
-static cudaError_t launch_attention_d(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &tk,
+                                      const CUtensorMap &tv, const __nv_bfloat16 *k,
                                       const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N,
                                       int nqb, int nkb, float scale_log2, const int32_t *counts,
                                       const int32_t *kv_index, const float *log_pi, int cap,
@@ -387,24 +495,25 @@ static cudaError_t launch_attention_d(const __nv_bfloat16 *q, const __nv_bfloat1
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     absa_attention_kernel<D, DENSE><<<(unsigned)(BH * nqb), kAttnThreads, smem, stream>>>(
-        q, k, v, o, N, nqb, nkb, scale_log2, counts, kv_index, log_pi, cap, status);
+        tq, tk, tv, k, v, o, N, nqb, nkb, scale_log2, counts, kv_index, log_pi, cap, status);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attention(bool dense, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+cudaError_t launch_attention(bool dense, const CUtensorMap &tq, const CUtensorMap &tk,
+                             const CUtensorMap &tv, const __nv_bfloat16 *k,
                              const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N, int nqb,
                              int nkb, int d, float softmax_scale, const int32_t *counts,
                              const int32_t *kv_index, const float *log_pi, int cap,
                              int32_t *status, cudaStream_t stream) {
     const float sl2 = softmax_scale * kLog2e;
     if (d == 64)
-        return dense ? launch_attention_d<64, true>(q, k, v, o, BH, N, nqb, nkb, sl2, counts,
+        return dense ? launch_attention_d<64, true>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
                                                     kv_index, log_pi, cap, status, stream)
-                     : launch_attention_d<64, false>(q, k, v, o, BH, N, nqb, nkb, sl2, counts,
+                     : launch_attention_d<64, false>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
                                                      kv_index, log_pi, cap, status, stream);
-    return dense ? launch_attention_d<128, true>(q, k, v, o, BH, N, nqb, nkb, sl2, counts,
+    return dense ? launch_attention_d<128, true>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
                                                  kv_index, log_pi, cap, status, stream)
-                 : launch_attention_d<128, false>(q, k, v, o, BH, N, nqb, nkb, sl2, counts,
+                 : launch_attention_d<128, false>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
                                                   kv_index, log_pi, cap, status, stream);
 }
 

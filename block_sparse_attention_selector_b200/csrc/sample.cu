@@ -34,7 +34,7 @@ __device__ __forceinline__ bool draw_taken(uint32_t u, uint64_t R, uint64_t rq) 
     return lhs_hi < rhs_hi || (lhs_hi == rhs_hi && lhs_lo < rhs_lo);
 }
 
-constexpr int kSampleThreads = 512;
+constexpr int kSampleThreads = 256;
 constexpr int kSampleWarps = kSampleThreads / 32;
 
 // Block-wide sum of a u64 and an int; result broadcast to every thread.
@@ -60,15 +60,20 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
     }
 }
 
-// One CTA per plan row (b,h,qb).  The score row is staged in shared memory
-// (4 bytes per key block) with one capped flag byte per block.
+// One CTA per plan row (b,h,qb).  Key blocks are handled in groups of 32 (one
+// per lane); warp w owns a contiguous run of groups, so the taken blocks of
+// warp w all precede those of warp w+1 and one scan of the 8 warp counts
+// places every entry.  Shared memory: q_j - 1 as u32 per block, plus one
+// capped word and one taken word (ballots) per group.
 __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
     uint64_t *__restrict__ r_R, int32_t *status) {
-    extern __shared__ __align__(16) uint8_t samp_smem[];
-    float *s = reinterpret_cast<float *>(samp_smem);
-    uint8_t *capped = samp_smem + (((size_t)nkb * 4 + 15) & ~(size_t)15);
+    extern __shared__ __align__(16) uint32_t samp_smem[];
+    const int ngroups = (nkb + 31) >> 5;
+    uint32_t *qm1 = samp_smem;                      // [ngroups*32]
+    uint32_t *capw = samp_smem + ngroups * 32;      // [ngroups]
+    uint32_t *takew = capw + ngroups;               // [ngroups]
     __shared__ uint64_t red_a[kSampleWarps];
     __shared__ int red_b[kSampleWarps];
     __shared__ int warp_cnt[kSampleWarps];
@@ -93,30 +98,46 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         return;
     }
 
+    const int per_warp = (ngroups + kSampleWarps - 1) / kSampleWarps;
+    const int g0 = warp * per_warp;
+    const int g1 = min(ngroups, g0 + per_warp);
+
+    // quantise once; R = sum of all q_j
     uint64_t R = 0;
     int dummy = 0;
-    for (int j = tid; j < nkb; j += kSampleThreads) {
-        const float v = __ldg(srow + j);
-        s[j] = v;
-        capped[j] = 0;
-        R += quantise_score(v);
+    for (int g = g0; g < g1; ++g) {
+        const int j = g * 32 + lane;
+        uint64_t qj = 0;
+        if (j < nkb) {
+            qj = quantise_score(__ldg(srow + j));
+            qm1[j] = (uint32_t)(qj - 1);
+        }
+        R += qj;
+        if (lane == 0) capw[g] = 0;
     }
-    block_sum2(R, dummy, red_a, red_b);  // also orders the shared-memory fill
+    block_sum2(R, dummy, red_a, red_b);
 
-    // capping fixed point: mark with (r, R), then recompute R over the rest
+    // capping fixed point: mark with (r, R), then the rest's sum is the next R
     int n_capped = 0;
     uint64_t r = (uint64_t)n;
     for (;;) {
         uint64_t rest = 0;
         int grew = 0;
-        for (int j = tid; j < nkb; j += kSampleThreads) {
-            if (capped[j]) continue;
-            const uint64_t qj = quantise_score(s[j]);
-            if (r * qj >= R) {
-                capped[j] = 1;
-                grew += 1;
-            } else {
-                rest += qj;
+        for (int g = g0; g < g1; ++g) {
+            const int j = g * 32 + lane;
+            const uint32_t word = capw[g];
+            bool newcap = false;
+            if (j < nkb && !((word >> lane) & 1u)) {
+                const uint64_t qj = (uint64_t)qm1[j] + 1;
+                if (r * qj >= R)
+                    newcap = true;
+                else
+                    rest += qj;
+            }
+            const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
+            if (nb) {
+                if (lane == 0) capw[g] = word | nb;
+                grew += lane == 0 ? __popc(nb) : 0;
             }
         }
         block_sum2(rest, grew, red_a, red_b);
@@ -125,56 +146,64 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         r = (uint64_t)(n - n_capped);
         R = rest;
     }
-    __syncthreads();
 
-    // Poisson draws and ascending compaction, 512 blocks per round
-    int base = 0;
+    // Poisson draws: one taken word per group
     const uint64_t ctr0 = (uint64_t)row * (uint64_t)nkb;
-    for (int j0 = 0; j0 < nkb; j0 += kSampleThreads) {
-        const int j = j0 + tid;
+    int taken = 0;
+    for (int g = g0; g < g1; ++g) {
+        const int j = g * 32 + lane;
         bool take = false;
-        float lp = 0.f;
         if (j < nkb) {
-            if (capped[j]) {
+            if ((capw[g] >> lane) & 1u) {
                 take = true;
             } else {
-                const uint64_t rq = r * quantise_score(s[j]);
+                const uint64_t rq = r * ((uint64_t)qm1[j] + 1);
                 take = draw_taken(draw_u32(seed, ctr0 + (uint64_t)j), R, rq);
-                if (take) lp = (float)log((double)rq / (double)R);
             }
         }
-        const uint32_t ballot = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) warp_cnt[warp] = __popc(ballot);
-        __syncthreads();
-        int before = 0, total = 0;
+        const uint32_t tw = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) takew[g] = tw;
+        taken += __popc(tw);
+    }
+    if (lane == 0) warp_cnt[warp] = taken;
+    __syncthreads();
+    int pos = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < kSampleWarps; ++w) {
-            const int c = warp_cnt[w];
-            before += w < warp ? c : 0;
-            total += c;
-        }
-        if (take) {
-            const int pos = base + before + __popc(ballot & ((1u << lane) - 1u));
-            if (pos < cap) {
-                idx_row[pos] = j;
-                lp_row[pos] = lp;
+    for (int w = 0; w < kSampleWarps; ++w) {
+        const int c = warp_cnt[w];
+        pos += w < warp ? c : 0;
+        total += c;
+    }
+    // ascending compaction of this warp's run
+    const uint32_t below = (1u << lane) - 1u;
+    for (int g = g0; g < g1 && pos < cap; ++g) {
+        const uint32_t tw = takew[g];
+        if ((tw >> lane) & 1u) {
+            const int j = g * 32 + lane;
+            const int p = pos + __popc(tw & below);
+            if (p < cap) {
+                idx_row[p] = j;
+                float lp = 0.f;
+                if (!((capw[g] >> lane) & 1u))
+                    lp = (float)log((double)(r * ((uint64_t)qm1[j] + 1)) / (double)R);
+                lp_row[p] = lp;
             }
         }
-        base += total;
-        __syncthreads();
+        pos += __popc(tw);
     }
     if (tid == 0) {
-        counts[row] = min(base, cap);
+        counts[row] = min(total, cap);
         r_R[2 * row] = r;
         r_R[2 * row + 1] = R;
-        if (base > cap) atomicOr(status, ABSA_DEVFLAG_OVERFLOW);
+        if (total > cap) atomicOr(status, ABSA_DEVFLAG_OVERFLOW);
     }
 }
 
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
                           int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
                           uint64_t *r_R, int32_t *status, cudaStream_t stream) {
-    const int smem = (int)((((size_t)nkb * 4 + 15) & ~(size_t)15) + (size_t)nkb + 16);
+    const int ngroups = (nkb + 31) / 32;
+    const int smem = (ngroups * 32 + 2 * ngroups) * 4;
     cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

@@ -65,9 +65,23 @@ __global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__r
 // widened to fp32 in shared memory (rows padded to D+1 words so that thread i
 // reading row i is bank-conflict free).  fp32 arithmetic in a fixed order:
 //  assignment (thread i): dist_c = sum over ascending e of fma(x-mu, x-mu, .),
-//                         argmin with ties to the lowest c;
-//  update     (thread e): member sums over ascending i, mu = sum / count
-//                         (IEEE division); an empty cluster keeps mu.
+//                         two clusters per packed f32x2 instruction (each lane
+//                         rounds exactly like the scalar operation), argmin
+//                         with ties to the lowest c;
+//  update     (thread e): member lists built by a stable counting sort, member
+//                         sums over ascending i, mu = sum / count (IEEE
+//                         division); an empty cluster keeps mu.
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     const __nv_bfloat16 *__restrict__ q, int N, int nqb, int iters, float *__restrict__ mu_out,
@@ -76,13 +90,14 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     constexpr int NC = 8;
     constexpr int XS = D + 1;
     extern __shared__ __align__(16) float kms[];
-    float *xs = kms;                    // [128][D+1]
-    float *mut = kms + 128 * XS;        // [D][8] centroids, transposed
+    float *xs = kms;                                   // [128][D+1]
+    float *mut = kms + 128 * XS;                       // [D][8] centroids, transposed
     int *asg = reinterpret_cast<int *>(mut + D * NC);  // [128]
-    int *cnt_s = asg + 128;             // [8]
+    int *cnt_s = asg + 128;                            // [8]
+    int *mlist = cnt_s + 8;                            // [8][128] member lists
 
     const int tid = threadIdx.x;
-    const int64_t row = blockIdx.x;     // (b*H + h)*nqb + qb
+    const int64_t row = blockIdx.x;  // (b*H + h)*nqb + qb
     const int64_t bh = row / nqb;
     const int qb = (int)(row % nqb);
     const int m = min(128, N - qb * 128);
@@ -107,67 +122,56 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     }
     __syncthreads();
 
-    int cnt[NC];
     for (int it = 0; it < iters; ++it) {
         if (tid < m) {
-            float dist[NC];
-#pragma unroll
-            for (int c = 0; c < NC; ++c) dist[c] = 0.f;
+            uint64_t dist[NC / 2] = {0, 0, 0, 0};  // (+0.f, +0.f) pairs
             const float *xr = xs + tid * XS;
 #pragma unroll 4
             for (int e = 0; e < D; ++e) {
-                const float xe = xr[e];
-                const float4 m0 = *reinterpret_cast<const float4 *>(mut + e * NC);
-                const float4 m1 = *reinterpret_cast<const float4 *>(mut + e * NC + 4);
-                const float mc[NC] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                const uint32_t xb = __float_as_uint(xr[e]);
+                const uint64_t x2 = (uint64_t)xb | ((uint64_t)xb << 32);
+                const ulonglong2 m01 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC);
+                const ulonglong2 m45 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC + 4);
+                const uint64_t mc[NC / 2] = {m01.x, m01.y, m45.x, m45.y};
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    const float diff = __fsub_rn(xe, mc[c]);
-                    dist[c] = __fmaf_rn(diff, diff, dist[c]);
+                for (int c = 0; c < NC / 2; ++c) {
+                    const uint64_t diff = f32x2_sub(x2, mc[c]);
+                    dist[c] = f32x2_fma(diff, diff, dist[c]);
                 }
             }
             int best = 0;
-            float bd = dist[0];
+            float bd = __uint_as_float((uint32_t)dist[0]);
 #pragma unroll
-            for (int c = 1; c < NC; ++c)
-                if (dist[c] < bd) {
-                    bd = dist[c];
+            for (int c = 1; c < NC; ++c) {
+                const float dc = __uint_as_float((uint32_t)(dist[c >> 1] >> (32 * (c & 1))));
+                if (dc < bd) {
+                    bd = dc;
                     best = c;
                 }
+            }
             asg[tid] = best;
         }
         __syncthreads();
-        {
-            float acc[NC];
-#pragma unroll
+        if (tid < NC) {  // stable counting sort: members of cluster tid, ascending i
+            int n = 0;
+            for (int i = 0; i < m; ++i)
+                if (asg[i] == tid) mlist[tid * 128 + n++] = i;
+            cnt_s[tid] = n;
+        }
+        __syncthreads();
+        if (tid < D) {
+#pragma unroll 1
             for (int c = 0; c < NC; ++c) {
-                acc[c] = 0.f;
-                cnt[c] = 0;
-            }
-            const int e = tid < D ? tid : 0;
-            for (int i = 0; i < m; ++i) {
-                const int a = asg[i];
-                const float xv = xs[i * XS + e];
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    if (a == c) {
-                        acc[c] = __fadd_rn(acc[c], xv);
-                        cnt[c] += 1;
-                    }
-            }
-            if (tid < D) {
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    if (cnt[c] > 0) mut[tid * NC + c] = __fdiv_rn(acc[c], (float)cnt[c]);
+                const int n = cnt_s[c];
+                if (n == 0) continue;
+                const int *ml = mlist + c * 128;
+                float acc = 0.f;
+                for (int t = 0; t < n; ++t) acc = __fadd_rn(acc, xs[ml[t] * XS + tid]);
+                mut[tid * NC + c] = __fdiv_rn(acc, (float)n);
             }
         }
         __syncthreads();
     }
-    if (tid == 0) {
-#pragma unroll
-        for (int c = 0; c < NC; ++c) cnt_s[c] = cnt[c];
-    }
-    __syncthreads();
     if (tid < NC) w_out[row * NC + tid] = __fdiv_rn((float)cnt_s[tid], (float)m);
     for (int idx = tid; idx < NC * D; idx += 128) {
         const int c = idx / D, e = idx % D;
@@ -421,7 +425,7 @@ template <int D>
 static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int iters,
                                    float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
                                    uint8_t *assign, cudaStream_t stream) {
-    const int smem = (128 * (D + 1) + D * 8) * 4 + 136 * 4;
+    const int smem = (128 * (D + 1) + D * 8) * 4 + (128 + 8 + 8 * 128) * 4;
     cudaError_t e = cudaFuncSetAttribute(absa_kmeans_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
