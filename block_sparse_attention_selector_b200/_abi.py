@@ -27,7 +27,10 @@ EXPORTED = (
     "absa_version", "absa_status_string", "absa_check_params", "absa_plan_capacity",
     "absa_workspace_bytes", "absa_select_scores", "absa_sample_plan", "absa_select_plan",
     "absa_sparse_attention", "absa_dense_reference", "absa_plan_check",
+    "absa_select_scores_static",
 )
+
+ABSA_STATIC_SCRATCH_BYTES = 64 << 20
 
 
 class absa_params(ctypes.Structure):
@@ -92,6 +95,8 @@ def lib():
         L.absa_dense_reference.restype = st
         L.absa_plan_check.argtypes = [Q, vp]
         L.absa_plan_check.restype = st
+        L.absa_select_scores_static.argtypes = [P, vp, vp, vp, vp]
+        L.absa_select_scores_static.restype = st
         _lib = L
     return _lib
 
@@ -145,3 +150,8 @@ def absa_dense_reference(p, q, k, v, o, status, stream):
 
 def absa_plan_check(plan, stream):
     return lib().absa_plan_check(ctypes.byref(plan), stream)
+
+
+def absa_select_scores_static(p, q, k, scores, stream):
+    """Selector scores with the library's built-in scratch (no workspace argument)."""
+    return lib().absa_select_scores_static(ctypes.byref(p), q, k, scores, stream)

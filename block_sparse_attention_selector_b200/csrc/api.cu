@@ -219,9 +219,42 @@ absa_status sample_plan_impl(const absa_params *p, const float *scores, const ab
     return from_cuda(e);
 }
 
+// Built-in workspace of absa_select_scores_static: one copy per device for as
+// long as the library is loaded.  Host code must not take its address
+// directly (the name is a host-side stand-in); static_scratch() resolves the
+// device address once per device.
+static __device__ __align__(256) uint8_t g_static_scratch[ABSA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_static_scratch on the current device (nullptr on error).
+void *static_scratch() {
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
+
+absa_status absa_select_scores_static(const absa_params *p, const void *q, const void *k,
+                                      float *scores, void *stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (ws_layout(p).total > ABSA_STATIC_SCRATCH_BYTES) return ABSA_ERR_WORKSPACE;
+    void *ws = static_scratch();
+    if (!ws) return ABSA_ERR_CUDA;
+    return select_scores_impl(p, q, k, scores, ws, ABSA_STATIC_SCRATCH_BYTES, nullptr, stream);
+}
 
 absa_status absa_select_scores(const absa_params *p, const void *q, const void *k, float *scores,
                                void *ws, size_t ws_bytes, void *stream) {

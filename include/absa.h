@@ -158,6 +158,34 @@ absa_status absa_sparse_attention(const absa_params *p, const void *q, const voi
 absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,
                                  const void *v, void *o, int32_t *status, void *stream);
 
+/* Size of the library's built-in scratch array used by
+ * absa_select_scores_static (bytes). */
+#define ABSA_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* Allocation-free variant of absa_select_scores (no counterpart on the
+ * pages: a library-interface addition).  It computes exactly what
+ * absa_select_scores computes, but takes its workspace from a 64 MiB array
+ * compiled into the library instead of a caller buffer, so callers that have
+ * no way to obtain device memory beyond their own inputs and outputs can
+ * still run the selector: plugin hosts that hand a plugin only its tensors,
+ * or code that runs under a memory manager it cannot call into.  The call
+ * itself never allocates or frees device memory.
+ *  - Limit: p must need at most ABSA_STATIC_SCRATCH_BYTES of workspace
+ *    (absa_workspace_bytes(p)); larger problems return ABSA_ERR_WORKSPACE
+ *    before any work is enqueued.
+ *  - The array exists once per GPU for as long as the library is loaded in
+ *    the process; the first call on a device looks up its device address
+ *    (with that device current), so make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the same array and leaves its contents
+ *    behind; nothing in it has to start at zero (each call writes every
+ *    region before reading it).  Calls that can run at the same time on one
+ *    GPU (different streams, or different host threads) race on the array:
+ *    serialise them.
+ * Arguments, layout and other errors as absa_select_scores. */
+absa_status absa_select_scores_static(const absa_params *p, const void *q, const void *k,
+                                      float *scores, void *stream);
+
 /* Synchronise `stream`, read plan->status and map it to a status code
  * (TIMEOUT > BAD_PLAN > OVERFLOW > OK).  Does not clear the word. */
 absa_status absa_plan_check(const absa_plan *plan, void *stream);
