@@ -75,12 +75,27 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 
 // Wait for the phase with the given parity.  Returns false (after setting the
 // timeout flag in *status and *abort) if it does not complete within about
-// kWaitLimitCycles, or if another thread of the CTA already gave up.  The
-// clock and the abort flag are read once every 16 sleeps so that waiting
-// warps take almost no issue slots.
+// kWaitLimitCycles, or if another thread of the CTA already gave up.  After a
+// short poll the thread sleeps between checks; the clock and the abort flag
+// are read once every 16 sleeps so that waiting warps take few issue slots.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
                                           volatile int *abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // short non-blocking poll first: most waits end within a few hundred cycles
+    // and a sleeping thread wakes up late
+    for (int i = 0; i < 64; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;

@@ -7,17 +7,17 @@
 // full-size tensor-core tiles, tokens are not permuted (third paragraph).
 //
 // Kernel design (one CTA per (b, h, 128-query block), 512 threads):
-//   warps 0-7   softmax, two warpgroups: warpgroup g handles columns
-//               64g..64g+63 of each S tile for all 128 rows (thread = TMEM
-//               lane = query row); the row max is exchanged through shared
-//               memory; warpgroup g rescales and stores output columns
-//               (d/2)g .. (d/2)g + d/2 - 1
+//   warps 0-7   softmax, two warpgroups: warpgroup g runs an independent
+//               online softmax over columns 64g..64g+63 of every S tile
+//               (thread = TMEM lane = query row) with its own accumulator
+//               O_g += P_g V_g; the halves are merged in the epilogue
 //   warps 8-14  loaders: TMA gathers of 32 blocks (= 128 key rows) per tile
 //               into SW128 shared-memory tiles, K and V in separate 2-stage
 //               rings, plus the tile's per-column logit bias
 //   warp 15     TMEM owner and MMA issuer (one thread):
 //              S_j = Q K_j^T  -> TMEM (two 128-column buffers)
-//              O  += P_j V_j  -> TMEM (D columns), P_j bf16 in shared memory
+//              O_g += P_j[:, 64g..] V_j[64g.., :] -> TMEM (two D-column
+//              accumulators), P_j bf16 in shared memory
 // Softmax works in the exp2 domain: x = log2(e) * scale * (q.k) + bias with
 // bias = -log2(pi) for a valid token and -inf for padding; row maxima are
 // updated lazily (O is rescaled only when the max grows by more than 2^8), and
@@ -37,7 +37,7 @@ struct AttnSmem {
     static constexpr int kVOff = kKOff + 2 * kKVBytes;         // [2] stages
     static constexpr int kPOff = kVOff + 2 * kKVBytes;         // 128 x 128 bf16
     static constexpr int kBiasOff = kPOff + 2 * kTile;         // [2][128] f32
-    static constexpr int kRedOff = kBiasOff + 2 * 128 * 4;    // [2][2][128] f32 exchange
+    static constexpr int kRedOff = kBiasOff + 2 * 128 * 4;    // [2][2][128] f32 final merge
     static constexpr int kBarOff = kRedOff + 4 * 128 * 4;
     static constexpr int kBytes = kBarOff + 24 * 8;
     // keep one CTA per SM so that the 512-column TMEM allocation never waits
@@ -83,13 +83,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     uint64_t *v_empty = bars + 7;  // [2]
     uint64_t *s_full = bars + 9;   // [2]
     uint64_t *s_free = bars + 11;  // [2]
-    uint64_t *p_full = bars + 13;
-    uint64_t *p_free = bars + 14;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 16);
-    float *red = reinterpret_cast<float *>(sm + S::kRedOff);  // [parity][half][row]
-    uint64_t *xchg = bars + 17;     // [2] row-max exchange of the two softmax warpgroups
-    uint64_t *xchg_end = bars + 19; // row-sum exchange before the epilogue
+    uint64_t *p_full = bars + 13;  // [2] per column half
+    uint64_t *p_free = bars + 15;  // [2] per column half
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
+    float *red = reinterpret_cast<float *>(sm + S::kRedOff);  // [max|sum][half][row]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -108,11 +106,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             mbar_init(s_full + s, 1);
             mbar_init(s_free + s, kSoftmaxWarps);
         }
-        mbar_init(p_full, kSoftmaxWarps);
-        mbar_init(p_free, 1);
-        mbar_init(xchg, kSoftmaxWarps);
-        mbar_init(xchg + 1, kSoftmaxWarps);
-        mbar_init(xchg_end, kSoftmaxWarps);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(p_full + h, kSoftmaxWarps / 2);
+            mbar_init(p_free + h, 1);
+        }
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -146,7 +143,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_o = tmem + 256;
+    const uint32_t tmem_o = tmem + 256;  // O_h at tmem_o + 128 h (h = column half)
 
     if (warp >= kLoadWarp && warp < kLoadWarp + kLoadWarps) {
         // ------------------------------------------------------------ loaders
@@ -264,12 +261,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             const uint32_t q_s = smem_u32(sm + S::kQOff);
             const uint32_t p_s = smem_u32(sm + S::kPOff);
             bool ok = mbar_wait(q_full, 0, status, abort_flag);
-            int js = 0, jp = 0;  // next S tile, next PV tile
+            int js = 0;            // next S tile
+            int jp[2] = {0, 0};    // next PV tile of each column half
             long long t0 = clock64();
             uint32_t spins = 0;
-            while (ok && jp < T) {
+            while (ok && (jp[0] < T || jp[1] < T)) {
                 bool progressed = false;
-                if (js < T && js < jp + 2) {
+                if (js < T && js < min(jp[0], jp[1]) + 2) {
                     const int st = js & 1;
                     if (mbar_try_wait(k_full + st, (js >> 1) & 1) &&
                         (js < 2 || mbar_try_wait(s_free + st, ((js - 2) >> 1) & 1))) {
@@ -288,23 +286,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                         progressed = true;
                     }
                 }
-                if (jp < js) {
-                    const int st = jp & 1;
-                    if (mbar_try_wait(p_full, jp & 1) && mbar_try_wait(v_full + st, (jp >> 1) & 1)) {
-                        tc_fence_after();
-                        const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
 #pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint64_t a =
-                                sw128_desc(p_s + (ks >> 2) * S::kTile + (ks & 3) * 32, 16, 1024);
-                            const uint64_t bdesc = sw128_desc(v_s + ks * 2048, S::kTile, 1024);
-                            tc_mma_f16(tmem_o, a, bdesc, idesc_o, (jp > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        tc_commit(p_free);
-                        tc_commit(v_empty + st);
-                        ++jp;
-                        progressed = true;
+                for (int h = 0; h < 2; ++h) {
+                    const int j = jp[h];
+                    if (j >= js) continue;
+                    const int st = j & 1;
+                    if (!mbar_try_wait(p_full + h, j & 1) || !mbar_try_wait(v_full + st, (j >> 1) & 1))
+                        continue;
+                    tc_fence_after();
+                    // O_h += P[:, 64h .. 64h+63] V[64h .. 64h+63, :]
+                    const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t a = sw128_desc(p_s + h * S::kTile + ks * 32, 16, 1024);
+                        const uint64_t bdesc =
+                            sw128_desc(v_s + (64 * h + 16 * ks) * 128, S::kTile, 1024);
+                        tc_mma_f16(tmem_o + 128 * h, a, bdesc, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
                     }
+                    tc_commit(p_free + h);
+                    jp[h] = j + 1;
+                    if (jp[1 - h] > j) tc_commit(v_empty + st);  // both halves of tile j issued
+                    progressed = true;
                 }
                 if (progressed) {
                     spins = 0;
@@ -326,15 +328,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         }
     } else {
         // ------------------------------------------------------------- softmax
-        // warpgroup `half` handles columns 64*half .. 64*half+63 of every S
-        // tile and output columns (D/2)*half ..; thread = TMEM lane = row.
+        // Warpgroup `half` runs its own online softmax over columns
+        // 64*half .. 64*half+63 of every S tile, with its own running max,
+        // row sum and accumulator O_half (O_half += P_half V_half); the two
+        // halves are merged in the epilogue, so no per-tile exchange is
+        // needed.  Thread = TMEM lane = query row.
         const int half = warp >> 2;
         const int r = (warp & 3) * 32 + lane;  // query row = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t p_s = smem_u32(sm + S::kPOff) + half * S::kTile;
         const int cb = 64 * half;
-        constexpr int OC = D / 2;              // output columns of this half
-        const uint32_t o_cols = tmem_o + half * OC;
+        const uint32_t o_h = tmem_o + 128 * half + lane_base;
         float m_ref = -INFINITY, lsum = 0.f;
         bool ok = true;
         for (int j = 0; j < T; ++j) {
@@ -370,26 +374,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                     const int a = (i >> 2) & 3;
                     mx4[a] = fmaxf(mx4[a], fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
                 }
-            // row max over both halves: exchange through shared memory
-            float *rx = red + (j & 1) * 256;
-            rx[half * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xchg + (j & 1));
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(xchg + (j & 1), (j >> 1) & 1, status, abort_flag));
-            if (!ok) break;
-            const float tmax = fmaxf(rx[r], rx[128 + r]);
-            if (j == 0) m_ref = tmax;
-            const bool need = j > 0 && tmax > m_ref + kRescaleThreshold;
-            const bool any_need = __any_sync(0xffffffffu, need);
+            const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            // lazy max: keep the reference unless the tile exceeds it by 2^8;
+            // a half whose columns so far were all padding has m_ref = -inf
+            const bool need = tmax > m_ref + kRescaleThreshold || (m_ref == -INFINITY && tmax > -INFINITY);
+            const bool any_need = j > 0 && __any_sync(0xffffffffu, need);
             const float m_new = need ? tmax : m_ref;
-            const float alpha = ex2(m_ref - m_new);
+            const float alpha = m_ref == -INFINITY ? 0.f : ex2(m_ref - m_new);
             m_ref = m_new;
-            if (j >= 1) {  // PV of the previous tile is done: P buffer free, O stable
-                ok = __all_sync(0xffffffffu, mbar_wait(p_free, (j - 1) & 1, status, abort_flag));
+            if (j >= 1) {  // PV of this half's previous tile is done: P half free, O_half stable
+                ok = __all_sync(0xffffffffu, mbar_wait(p_free + half, (j - 1) & 1, status, abort_flag));
                 if (!ok) break;
             }
-            const float moff = -m_ref;
+            const float moff = m_ref == -INFINITY ? 0.f : -m_ref;
             float acc8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc8[i] = 0.f;
@@ -410,18 +407,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                                  : "memory");
                 }
             }
-            if (any_need) {  // lazy rescale of this half's output columns
+            if (any_need) {  // lazy rescale of O_half by exp2(m_old - m_new)
                 tc_fence_after();
                 lsum *= alpha;
 #pragma unroll
-                for (int ch = 0; ch < OC / 32; ++ch) {
+                for (int ch = 0; ch < D / 32; ++ch) {
                     uint32_t ov[32];
-                    tmem_ld32(o_cols + lane_base + ch * 32, ov);
+                    tmem_ld32(o_h + ch * 32, ov);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(o_cols + lane_base + ch * 32, ov);
+                    tmem_st32(o_h + ch * 32, ov);
                 }
                 tmem_wait_st();
             }
@@ -430,40 +427,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full + half);
         }
-        // epilogue: O / (sum over both halves) -> bf16, valid rows only
-        // (the parity buffer of tile T is free: its last readers passed tile T-1)
-        float *rs = red + (T & 1) * 256;
-        rs[half * 128 + r] = lsum;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(xchg_end);
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(xchg_end, 0, status, abort_flag));
-        const float ltot = rs[r] + rs[128 + r];
+        // epilogue: o = (O_0 a_0 + O_1 a_1) / (l_0 a_0 + l_1 a_1), a_h = 2^(m_h - max);
+        // warpgroup `half` writes output columns (D/2) half .. (D/2) half + D/2 - 1.
+        // Every softmax thread reaches this barrier exactly once.
+        red[half * 128 + r] = m_ref;
+        red[256 + half * 128 + r] = lsum;
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        const float m0 = red[r], m1 = red[128 + r];
+        const float mm = fmaxf(m0, m1);
+        const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+        const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
+        const float ltot = red[256 + r] * a0 + red[384 + r] * a1;
+        constexpr int OC = D / 2;
         __nv_bfloat16 *orow = o + (bh * N + (int64_t)qb * 128 + r) * D + half * OC;
         if (T > 0 && ok) {
-            ok = __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, status, abort_flag));
+            ok = __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, status, abort_flag) &&
+                                             mbar_wait(p_free + 1, (T - 1) & 1, status, abort_flag));
         }
         if (T > 0 && ok) {
             tc_fence_after();
             const float inv = 1.f / ltot;
+            const float c0 = a0 * inv, c1 = a1 * inv;
 #pragma unroll
             for (int ch = 0; ch < OC / 32; ++ch) {
-                uint32_t ov[32];
-                tmem_ld32(o_cols + lane_base + ch * 32, ov);
+                uint32_t o0[32], o1[32];
+                tmem_ld32(tmem_o + lane_base + half * OC + ch * 32, o0);
+                tmem_ld32(tmem_o + 128 + lane_base + half * OC + ch * 32, o1);
                 tmem_wait_ld();
                 if (r < m) {
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            f[e] = __uint_as_float(o0[8 * g + e]) * c0 +
+                                   __uint_as_float(o1[8 * g + e]) * c1;
                         uint4 u;
-                        u.x = pack_bf16x2(__uint_as_float(ov[8 * g + 0]) * inv,
-                                          __uint_as_float(ov[8 * g + 1]) * inv);
-                        u.y = pack_bf16x2(__uint_as_float(ov[8 * g + 2]) * inv,
-                                          __uint_as_float(ov[8 * g + 3]) * inv);
-                        u.z = pack_bf16x2(__uint_as_float(ov[8 * g + 4]) * inv,
-                                          __uint_as_float(ov[8 * g + 5]) * inv);
-                        u.w = pack_bf16x2(__uint_as_float(ov[8 * g + 6]) * inv,
-                                          __uint_as_float(ov[8 * g + 7]) * inv);
+                        u.x = pack_bf16x2(f[0], f[1]);
+                        u.y = pack_bf16x2(f[2], f[3]);
+                        u.z = pack_bf16x2(f[4], f[5]);
+                        u.w = pack_bf16x2(f[6], f[7]);
                         *reinterpret_cast<uint4 *>(orow + ch * 32 + 8 * g) = u;
                     }
                 }

@@ -7,7 +7,8 @@
 // Integer formulation (exact, so every ordering of the reductions gives the
 // same plan): q_j = max(1, floor(s_j 2^32)); capping fixed point on
 // (r, R) = (n - |C|, sum_{j not in C} q_j) with u64 block reductions; draw
-// u_j * R < (r q_j) 2^32 compared in 128 bits.
+// u_j * R < (r q_j) 2^32 compared exactly.  u_j is output ctr+1 of the
+// SplitMix64 generator started from state mix(seed), ctr = row * NKB + j.
 #include "absa_kernels.cuh"
 
 namespace absa {
@@ -19,19 +20,13 @@ __device__ __forceinline__ uint64_t quantise_score(float s) {
     return (uint64_t)x;                 // floor for x >= 1
 }
 
-__device__ __forceinline__ uint32_t draw_u32(uint64_t seed, uint64_t ctr) {
-    uint64_t z = splitmix64_mix(ctr + 0x9E3779B97F4A7C15ull);
-    z = splitmix64_mix(z ^ seed);
-    return (uint32_t)(z >> 32);
-}
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;  // SplitMix64 increment
 
-// u * R < rq * 2^32 in 128-bit arithmetic (u < 2^32, R and rq < 2^48).
-__device__ __forceinline__ bool draw_taken(uint32_t u, uint64_t R, uint64_t rq) {
-    const uint64_t lhs_lo = (uint64_t)u * R;
-    const uint64_t lhs_hi = __umul64hi((uint64_t)u, R);
-    const uint64_t rhs_lo = rq << 32;
-    const uint64_t rhs_hi = rq >> 32;
-    return lhs_hi < rhs_hi || (lhs_hi == rhs_hi && lhs_lo < rhs_lo);
+// u * R < rq * 2^32 exactly (u < 2^32, R < 2^48, rq < 2^48): with
+// R = Rh 2^32 + Rl, u R = (u Rh + hi32(u Rl)) 2^32 + lo32(u Rl), so the
+// comparison reduces to u Rh + hi32(u Rl) < rq.
+__device__ __forceinline__ bool draw_taken(uint32_t u, uint32_t Rh, uint32_t Rl, uint64_t rq) {
+    return (uint64_t)u * Rh + __umulhi(u, Rl) < rq;
 }
 
 constexpr int kSampleThreads = 256;
@@ -120,6 +115,7 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     // capping fixed point: mark with (r, R), then the rest's sum is the next R
     int n_capped = 0;
     uint64_t r = (uint64_t)n;
+    uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
     for (;;) {
         uint64_t rest = 0;
         int grew = 0;
@@ -128,11 +124,11 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
             const uint32_t word = capw[g];
             bool newcap = false;
             if (j < nkb && !((word >> lane) & 1u)) {
-                const uint64_t qj = (uint64_t)qm1[j] + 1;
-                if (r * qj >= R)
+                const uint32_t q1 = qm1[j];
+                if ((uint64_t)r32 * q1 + r32 >= R)  // r * q_j
                     newcap = true;
                 else
-                    rest += qj;
+                    rest += (uint64_t)q1 + 1;
             }
             const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
             if (nb) {
@@ -144,11 +140,14 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         if (grew == 0) break;
         n_capped += grew;
         r = (uint64_t)(n - n_capped);
+        r32 = (uint32_t)r;
         R = rest;
     }
 
-    // Poisson draws: one taken word per group
-    const uint64_t ctr0 = (uint64_t)row * (uint64_t)nkb;
+    // Poisson draws: one taken word per group; SplitMix64 state of block j is
+    // base + j * gamma with base = mix(seed) + (row * NKB + 1) * gamma
+    const uint64_t base = splitmix64_mix(seed) + ((uint64_t)row * (uint64_t)nkb + 1) * kGamma;
+    const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
     int taken = 0;
     for (int g = g0; g < g1; ++g) {
         const int j = g * 32 + lane;
@@ -157,8 +156,9 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
             if ((capw[g] >> lane) & 1u) {
                 take = true;
             } else {
-                const uint64_t rq = r * ((uint64_t)qm1[j] + 1);
-                take = draw_taken(draw_u32(seed, ctr0 + (uint64_t)j), R, rq);
+                const uint64_t rq = (uint64_t)r32 * qm1[j] + r32;
+                const uint32_t u = (uint32_t)(splitmix64_mix(base + (uint64_t)j * kGamma) >> 32);
+                take = draw_taken(u, Rh, Rl, rq);
             }
         }
         const uint32_t tw = __ballot_sync(0xffffffffu, take);
@@ -174,22 +174,26 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         pos += w < warp ? c : 0;
         total += c;
     }
-    // ascending compaction of this warp's run
+    // ascending compaction of this warp's run (block ids only)
     const uint32_t below = (1u << lane) - 1u;
     for (int g = g0; g < g1 && pos < cap; ++g) {
         const uint32_t tw = takew[g];
         if ((tw >> lane) & 1u) {
-            const int j = g * 32 + lane;
             const int p = pos + __popc(tw & below);
-            if (p < cap) {
-                idx_row[p] = j;
-                float lp = 0.f;
-                if (!((capw[g] >> lane) & 1u))
-                    lp = (float)log((double)(r * ((uint64_t)qm1[j] + 1)) / (double)R);
-                lp_row[p] = lp;
-            }
+            if (p < cap) idx_row[p] = g * 32 + lane;
         }
         pos += __popc(tw);
+    }
+    __syncthreads();  // the block ids written above are visible to the whole CTA
+    // ln(pi) of the written entries, all lanes busy (the double-precision
+    // logarithm would otherwise run for a whole warp per taken lane)
+    const int written = min(total, cap);
+    for (int p = tid; p < written; p += kSampleThreads) {
+        const int j = idx_row[p];
+        float lp = 0.f;
+        if (!((capw[j >> 5] >> (j & 31)) & 1u))
+            lp = (float)log((double)((uint64_t)r32 * qm1[j] + r32) / (double)R);
+        lp_row[p] = lp;
     }
     if (tid == 0) {
         counts[row] = min(total, cap);

@@ -61,16 +61,17 @@ __global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__r
 
 // ------------------------------------------------------------------------ K2
 
-// One CTA (128 threads) per query block.  The block's m valid queries are
-// widened to fp32 in shared memory (rows padded to D+1 words so that thread i
-// reading row i is bank-conflict free).  fp32 arithmetic in a fixed order:
+// One CTA (128 threads) per query block.  fp32 arithmetic in a fixed order:
 //  assignment (thread i): dist_c = sum over ascending e of fma(x-mu, x-mu, .),
 //                         two clusters per packed f32x2 instruction (each lane
 //                         rounds exactly like the scalar operation), argmin
 //                         with ties to the lowest c;
-//  update     (thread e): member lists built by a stable counting sort, member
-//                         sums over ascending i, mu = sum / count (IEEE
-//                         division); an empty cluster keeps mu.
+//  update     (thread e): members of each cluster ranked in ascending i with
+//                         warp ballots, member sums over ascending i read from
+//                         the bf16 copy of the block in shared memory (no bank
+//                         conflicts: a warp reads 32 consecutive columns of one
+//                         row), mu = sum / count (IEEE division); an empty
+//                         cluster keeps mu.
 __device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -83,81 +84,103 @@ __device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c
 }
 
 template <int D>
+struct KmeansSmem {
+    static constexpr int kRow = D + 2;                  // bf16 row pitch: 4*(D/2+1) bytes, so
+                                                        // thread i reading row i is conflict-free
+    static constexpr int kX = 0;                        // bf16 [128][D+2]
+    static constexpr int kMu = kX + 128 * kRow * 2;     // f32 [D][8] (transposed)
+    static constexpr int kList = kMu + D * 8 * 4;       // i32 [8][128] member lists
+    static constexpr int kCnt = kList + 8 * 128 * 4;    // i32 [4 warps][8] + [8] totals
+    static constexpr int kBytes = kCnt + (4 * 8 + 8) * 4;
+};
+
+template <int D>
 __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     const __nv_bfloat16 *__restrict__ q, int N, int nqb, int iters, float *__restrict__ mu_out,
     __nv_bfloat16 *__restrict__ mu_hi, __nv_bfloat16 *__restrict__ mu_lo, float *__restrict__ w_out,
     uint8_t *__restrict__ assign_out) {
+    using S = KmeansSmem<D>;
     constexpr int NC = 8;
-    constexpr int XS = D + 1;
-    extern __shared__ __align__(16) float kms[];
-    float *xs = kms;                                   // [128][D+1]
-    float *mut = kms + 128 * XS;                       // [D][8] centroids, transposed
-    int *asg = reinterpret_cast<int *>(mut + D * NC);  // [128]
-    int *cnt_s = asg + 128;                            // [8]
-    int *mlist = cnt_s + 8;                            // [8][128] member lists
+    constexpr int CH = D / 8;  // 16-byte chunks per row
+    extern __shared__ __align__(16) uint8_t kms[];
+    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(kms + S::kX);
+    float *mut = reinterpret_cast<float *>(kms + S::kMu);
+    int *mlist = reinterpret_cast<int *>(kms + S::kList);
+    int *wcnt = reinterpret_cast<int *>(kms + S::kCnt);  // [warp][c]
+    int *cnt_s = wcnt + 4 * NC;                          // [c]
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = blockIdx.x;  // (b*H + h)*nqb + qb
     const int64_t bh = row / nqb;
     const int qb = (int)(row % nqb);
     const int m = min(128, N - qb * 128);
     const __nv_bfloat16 *src = q + (bh * N + (int64_t)qb * 128) * D;
 
-    constexpr int CH = D / 8;
-    for (int idx = tid; idx < m * CH; idx += 128) {
-        const int r = idx / CH, c = idx % CH;
-        uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)r * D + c * 8));
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(h2[e]);
-            xs[r * XS + c * 8 + 2 * e] = f.x;
-            xs[r * XS + c * 8 + 2 * e + 1] = f.y;
+    constexpr int XR = S::kRow;
+    {
+        const uint32_t *src32 = reinterpret_cast<const uint32_t *>(src);
+        uint32_t *xs32 = reinterpret_cast<uint32_t *>(xs);
+        for (int idx = tid; idx < m * (D / 2); idx += 128) {
+            const int r = idx / (D / 2), w = idx % (D / 2);
+            xs32[r * (XR / 2) + w] = __ldg(src32 + idx);
         }
     }
     __syncthreads();
     for (int idx = tid; idx < NC * D; idx += 128) {
         const int c = idx / D, e = idx % D;
-        mut[e * NC + c] = xs[((c * m) / NC) * XS + e];
+        mut[e * NC + c] = __bfloat162float(xs[((c * m) / NC) * XR + e]);
     }
     __syncthreads();
 
     for (int it = 0; it < iters; ++it) {
+        int a = 0;
         if (tid < m) {
             uint64_t dist[NC / 2] = {0, 0, 0, 0};  // (+0.f, +0.f) pairs
-            const float *xr = xs + tid * XS;
+            const uint32_t *xrow = reinterpret_cast<const uint32_t *>(xs + tid * XR);
 #pragma unroll 4
-            for (int e = 0; e < D; ++e) {
-                const uint32_t xb = __float_as_uint(xr[e]);
-                const uint64_t x2 = (uint64_t)xb | ((uint64_t)xb << 32);
-                const ulonglong2 m01 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC);
-                const ulonglong2 m45 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC + 4);
-                const uint64_t mc[NC / 2] = {m01.x, m01.y, m45.x, m45.y};
+            for (int e2 = 0; e2 < D / 2; ++e2) {
+                const uint32_t pair = xrow[e2];
 #pragma unroll
-                for (int c = 0; c < NC / 2; ++c) {
-                    const uint64_t diff = f32x2_sub(x2, mc[c]);
-                    dist[c] = f32x2_fma(diff, diff, dist[c]);
+                for (int h = 0; h < 2; ++h) {
+                    const int e = 2 * e2 + h;
+                    const uint32_t xb = h ? (pair & 0xFFFF0000u) : (pair << 16);
+                    const uint64_t x2 = (uint64_t)xb | ((uint64_t)xb << 32);
+                    const ulonglong2 m01 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC);
+                    const ulonglong2 m45 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC + 4);
+                    const uint64_t mc[NC / 2] = {m01.x, m01.y, m45.x, m45.y};
+#pragma unroll
+                    for (int c = 0; c < NC / 2; ++c) {
+                        const uint64_t diff = f32x2_sub(x2, mc[c]);
+                        dist[c] = f32x2_fma(diff, diff, dist[c]);
+                    }
                 }
             }
-            int best = 0;
             float bd = __uint_as_float((uint32_t)dist[0]);
 #pragma unroll
             for (int c = 1; c < NC; ++c) {
                 const float dc = __uint_as_float((uint32_t)(dist[c >> 1] >> (32 * (c & 1))));
                 if (dc < bd) {
                     bd = dc;
-                    best = c;
+                    a = c;
                 }
             }
-            asg[tid] = best;
+        }
+        // rank of query tid among the members of its cluster (ascending i)
+        const bool valid = tid < m;
+        uint32_t my_ballot = 0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const uint32_t bal = __ballot_sync(0xffffffffu, valid && a == c);
+            if (lane == 0) wcnt[warp * NC + c] = __popc(bal);
+            if (a == c) my_ballot = bal;
         }
         __syncthreads();
-        if (tid < NC) {  // stable counting sort: members of cluster tid, ascending i
-            int n = 0;
-            for (int i = 0; i < m; ++i)
-                if (asg[i] == tid) mlist[tid * 128 + n++] = i;
-            cnt_s[tid] = n;
+        if (valid) {
+            int pos = __popc(my_ballot & ((1u << lane) - 1u));
+            for (int w = 0; w < warp; ++w) pos += wcnt[w * NC + a];
+            mlist[a * 128 + pos] = tid;
         }
+        if (tid < NC) cnt_s[tid] = wcnt[tid] + wcnt[NC + tid] + wcnt[2 * NC + tid] + wcnt[3 * NC + tid];
         __syncthreads();
         if (tid < D) {
 #pragma unroll 1
@@ -166,7 +189,15 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
                 if (n == 0) continue;
                 const int *ml = mlist + c * 128;
                 float acc = 0.f;
-                for (int t = 0; t < n; ++t) acc = __fadd_rn(acc, xs[ml[t] * XS + tid]);
+                int t = 0;
+                for (; t + 4 <= n; t += 4) {  // loads ahead, adds in order
+                    const float x0 = __bfloat162float(xs[ml[t] * XR + tid]);
+                    const float x1 = __bfloat162float(xs[ml[t + 1] * XR + tid]);
+                    const float x2 = __bfloat162float(xs[ml[t + 2] * XR + tid]);
+                    const float x3 = __bfloat162float(xs[ml[t + 3] * XR + tid]);
+                    acc = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(acc, x0), x1), x2), x3);
+                }
+                for (; t < n; ++t) acc = __fadd_rn(acc, __bfloat162float(xs[ml[t] * XR + tid]));
                 mut[tid * NC + c] = __fdiv_rn(acc, (float)n);
             }
         }
@@ -182,7 +213,10 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
         mu_hi[o] = h;
         mu_lo[o] = __float2bfloat16_rn(v - __bfloat162float(h));
     }
-    assign_out[row * 128 + tid] = tid < m ? (uint8_t)asg[tid] : (uint8_t)255;
+    // final assignment: member lists of the last round
+    for (int c = 0; c < NC; ++c)
+        for (int t = tid; t < cnt_s[c]; t += 128) assign_out[row * 128 + mlist[c * 128 + t]] = (uint8_t)c;
+    if (tid >= m) assign_out[row * 128 + tid] = (uint8_t)255;
 }
 
 // ------------------------------------------------------------------------ K3
@@ -198,7 +232,10 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
 //   pass 2: D[j, (qb,c)] = kbar . mu   (A = key tile, B = centroids); the
 //           thread owning lane j forms s_j = sum_c exp2(scaled logit - L_c)
 //           for each of the 16 query blocks and stores it.
-// Warps: 0 TMA producer, 1 MMA issuer (+TMEM owner), 2..5 epilogue.
+// Warps: 0 TMA producer, 1 MMA issuer (+TMEM owner), 2..9 epilogue in two
+// warpgroups: warpgroup g takes columns 64g..64g+63 of every tile (pass 1:
+// its own online max/sum, merged with the other half once at the end; pass
+// 2: query blocks 8g..8g+7 of the group).
 template <int D>
 struct ScoreSmem {
     static constexpr int kRegions = D / 64;                 // 64-element SW128 regions
@@ -207,14 +244,15 @@ struct ScoreSmem {
     static constexpr int kKbBytes = 2 * kRegions * kTile;   // one stage, hi + lo
     static constexpr int kMuOff = 0;
     static constexpr int kKbOff = kMuBytes;
-    static constexpr int kLOff = kKbOff + 2 * kKbBytes;
-    static constexpr int kBarOff = kLOff + 128 * 4;
+    static constexpr int kLOff = kKbOff + 2 * kKbBytes;     // f32 [128] L per centroid row
+    static constexpr int kXOff = kLOff + 128 * 4;           // f32 [2][2][128] pass-1 halves
+    static constexpr int kBarOff = kXOff + 4 * 128 * 4;
     static constexpr int kBytes = kBarOff + 16 * 8 + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) absa_score_kernel(
+__global__ void __launch_bounds__(320, 1) absa_score_kernel(
     const __grid_constant__ CUtensorMap tm_kb_hi, const __grid_constant__ CUtensorMap tm_kb_lo,
     const __grid_constant__ CUtensorMap tm_mu_hi, const __grid_constant__ CUtensorMap tm_mu_lo,
     const float *__restrict__ w, float *__restrict__ scores, int nqb, int nkb, int groups,
@@ -247,7 +285,7 @@ __global__ void __launch_bounds__(192, 1) absa_score_kernel(
             mbar_init(kb_full + s, 1);
             mbar_init(kb_empty + s, 1);
             mbar_init(d_full + s, 1);
-            mbar_init(d_empty + s, 4);
+            mbar_init(d_empty + s, 8);
         }
         *abort_flag = 0;
         mbar_fence_init();
@@ -318,63 +356,75 @@ __global__ void __launch_bounds__(192, 1) absa_score_kernel(
             }
         }
     } else {
-        // epilogue: thread <-> TMEM lane (warps 2..5 own lane quarters 2,3,0,1)
+        // epilogue: thread <-> TMEM lane; warp w owns lane quarter w % 4
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;  // column half (warpgroup)
         const int lrow = quarter * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + half * 64;
+        float *xch = reinterpret_cast<float *>(sm + S::kXOff);  // [max|sum][half][row]
         bool ok = true;
-        // pass 1: online log-sum-exp over the key blocks of this centroid row
+        // pass 1: online log-sum-exp over this half's key blocks of the row
         float mx = -INFINITY, sum = 0.f;
         for (int t = 0; t < T && ok; ++t) {
             const int buf = t & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(d_full + buf, (t >> 1) & 1, status, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            uint32_t v[4][32];
+            uint32_t v[2][32];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
+            for (int ch = 0; ch < 2; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(d_empty + buf);
-            const int ncols = min(128, nkb - t * 128);
-            float tmax = -INFINITY;
+            const int ncols = min(64, nkb - t * 128 - half * 64);
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
+            for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (ch * 32 + i < ncols) tmax = fmaxf(tmax, __uint_as_float(v[ch][i]));
+                    if (ch * 32 + i < ncols) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(v[ch][i]));
+            const float tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             if (tmax > mx) {
                 sum *= ex2((mx - tmax) * scale_log2);
                 mx = tmax;
             }
             const float moff = -mx * scale_log2;
-            float acc = 0.f;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
+            for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     if (ch * 32 + i < ncols)
-                        acc += ex2(__fmaf_rn(__uint_as_float(v[ch][i]), scale_log2, moff));
-            sum += acc;
+                        a4[i & 3] += ex2(__fmaf_rn(__uint_as_float(v[ch][i]), scale_log2, moff));
+            sum += (a4[0] + a4[1]) + (a4[2] + a4[3]);
         }
+        // merge the two halves of each row (every epilogue thread passes here once)
+        xch[half * 128 + lrow] = mx;
+        xch[256 + half * 128 + lrow] = sum;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         {
+            const float m0 = xch[lrow], m1 = xch[128 + lrow];
+            const float mm = fmaxf(m0, m1);
+            const float s0 = xch[256 + lrow], s1 = xch[384 + lrow];
+            const float tot = (m0 == -INFINITY ? 0.f : s0 * ex2((m0 - mm) * scale_log2)) +
+                              (m1 == -INFINITY ? 0.f : s1 * ex2((m1 - mm) * scale_log2));
             const int qb = qb0 + (lrow >> 3);
             const float wc = qb < nqb ? w[(bh * nqb + qb) * 8 + (lrow & 7)] : 0.f;
-            const float lse2 = mx * scale_log2 + log2f(sum);
-            Ltab[lrow] = wc > 0.f ? lse2 - log2f(wc) : INFINITY;
+            const float lse2 = mm * scale_log2 + log2f(tot);
+            if (half == 0) Ltab[lrow] = wc > 0.f ? lse2 - log2f(wc) : INFINITY;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // pass 2: combine the 8 centroids of each query block for key block j = lane row
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        // pass 2: combine the 8 centroids of each of this half's query blocks
         for (int t = 0; t < T && ok; ++t) {
             const int g = T + t;
             const int buf = g & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(d_full + buf, (g >> 1) & 1, status, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            uint32_t v[4][32];
+            uint32_t v[2][32];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
+            for (int ch = 0; ch < 2; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -382,20 +432,20 @@ __global__ void __launch_bounds__(192, 1) absa_score_kernel(
             const int j = t * 128 + lrow;
             if (j < nkb) {
 #pragma unroll
-                for (int qbl = 0; qbl < 16; ++qbl) {
-                    const int qb = qb0 + qbl;
+                for (int qbl = 0; qbl < 8; ++qbl) {
+                    const int qb = qb0 + half * 8 + qbl;
                     if (qb >= nqb) continue;
-                    const float4 L0 = *reinterpret_cast<const float4 *>(Ltab + qbl * 8);
-                    const float4 L1 = *reinterpret_cast<const float4 *>(Ltab + qbl * 8 + 4);
+                    const float4 L0 = *reinterpret_cast<const float4 *>(Ltab + (half * 8 + qbl) * 8);
+                    const float4 L1 = *reinterpret_cast<const float4 *>(Ltab + (half * 8 + qbl) * 8 + 4);
                     const float Lc[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
-                    float s = 0.f;
+                    float s2[2] = {0.f, 0.f};
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const int col = qbl * 8 + c;
-                        s += ex2(__fmaf_rn(__uint_as_float(v[col >> 5][col & 31]), scale_log2,
-                                           -Lc[c]));
+                        s2[c & 1] += ex2(__fmaf_rn(__uint_as_float(v[col >> 5][col & 31]),
+                                                   scale_log2, -Lc[c]));
                     }
-                    scores[(bh * nqb + qb) * (int64_t)nkb + j] = s;
+                    scores[(bh * nqb + qb) * (int64_t)nkb + j] = s2[0] + s2[1];
                 }
             }
         }
@@ -425,7 +475,7 @@ template <int D>
 static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int iters,
                                    float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
                                    uint8_t *assign, cudaStream_t stream) {
-    const int smem = (128 * (D + 1) + D * 8) * 4 + (128 + 8 + 8 * 128) * 4;
+    const int smem = KmeansSmem<D>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(absa_kmeans_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -451,7 +501,7 @@ static cudaError_t launch_score_d(const CUtensorMap &a, const CUtensorMap &b, co
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int groups = (nqb + 15) / 16;
-    absa_score_kernel<D><<<(unsigned)(BH * groups), 192, smem, stream>>>(
+    absa_score_kernel<D><<<(unsigned)(BH * groups), 320, smem, stream>>>(
         a, b, c, dd, w, scores, nqb, nkb, groups, scale_log2, status);
     return cudaGetLastError();
 }

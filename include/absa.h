@@ -124,8 +124,9 @@ absa_status absa_select_scores(const absa_params *p, const void *q, const void *
  * negative -> 1, at most 2^32); from C = {} repeat r = n - |C|,
  * R = sum_{j not in C} q_j, C += {j : r*q_j >= R} until C is unchanged;
  * pi_j = 1 on C, r*q_j/R elsewhere, so sum pi = n exactly.  Poisson draws:
- * u_j = mix(mix(row*NKB + j + 0x9E3779B97F4A7C15) ^ seed) >> 32 with mix the
- * SplitMix64 output function and row = (b*H + h)*NQB + qb; block j is taken
+ * with ctr = row*NKB + j, row = (b*H + h)*NQB + qb, and mix the SplitMix64
+ * output function, u_j = mix(mix(seed) + (ctr+1)*0x9E3779B97F4A7C15) >> 32
+ * (output ctr+1 of SplitMix64 started from state mix(seed)); block j is taken
  * iff j in C or u_j * R < r*q_j * 2^32.  Taken blocks are written ascending
  * with log_pi = 0 (capped) or (float)ln((double)(r*q_j)/R).  n >= NKB takes
  * every block.  Resets plan->status first; a row with more than

@@ -199,8 +199,9 @@ uint64_t oracle_splitmix64_mix(uint64_t z)
 
 uint32_t oracle_draw_u32(uint64_t seed, uint64_t ctr)
 {
-    uint64_t z = oracle_splitmix64_mix(ctr + 0x9E3779B97F4A7C15ull);
-    z = oracle_splitmix64_mix(z ^ seed);
+    /* output number ctr+1 of SplitMix64 started from state key = mix(seed) */
+    uint64_t key = oracle_splitmix64_mix(seed);
+    uint64_t z = oracle_splitmix64_mix(key + (ctr + 1) * 0x9E3779B97F4A7C15ull);
     return (uint32_t)(z >> 32);
 }
 

@@ -76,8 +76,10 @@ int oracle_pi_solve(const float *s, int nkb, int64_t n, uint8_t *capped,
 uint64_t oracle_splitmix64_mix(uint64_t z);
 
 /* Counter-based uniform for the SIP draw of block j of row `row`:
- * ctr = row*nkb + j, z = mix(ctr + 0x9E3779B97F4A7C15), z = mix(z ^ seed),
- * u = z >> 32. */
+ * ctr = row*nkb + j; u = high 32 bits of output number ctr+1 of the
+ * SplitMix64 generator started from state key = mix(seed), i.e.
+ * u = mix(key + (ctr+1) * 0x9E3779B97F4A7C15) >> 32 (mod 2^64 arithmetic).
+ * mix(0) = 0, so seed 0 gives the published SplitMix64 stream from state 0. */
 uint32_t oracle_draw_u32(uint64_t seed, uint64_t ctr);
 
 /* SIP plan for one row (b,h,qb) whose flat index is `row`

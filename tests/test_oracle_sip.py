@@ -92,11 +92,23 @@ def test_splitmix64_published_outputs():
     assert got == [int(x, 16) for x in g["outputs_from_state_0"]]
 
 
-def test_draw_is_second_mix_of_seed_xor_first():
-    # u = mix(mix(ctr + gamma) ^ seed) >> 32; with seed 0 and ctr 0 this is
-    # mix(first reference output) >> 32
-    first = 0xE220A8397B1DCDAF
-    assert oracle.draw_u32(0, 0) == oracle.splitmix64_mix(first) >> 32
+def test_draws_with_seed_zero_are_the_published_splitmix64_stream():
+    # mix(0) = 0, so seed 0 draws are the high halves of SplitMix64 from state 0
+    with open(os.path.join(GOLDEN, "splitmix64_reference.json")) as f:
+        g = json.load(f)
+    for ctr, out in enumerate(g["outputs_from_state_0"]):
+        assert oracle.draw_u32(0, ctr) == int(out, 16) >> 32
+
+
+def test_draw_seed_selects_a_keyed_stream():
+    # seed s uses the stream started from mix(s): output ctr+1 of that stream
+    gamma = 0x9E3779B97F4A7C15
+    for seed in (1, 17, 2**63 + 5):
+        key = oracle.splitmix64_mix(seed)
+        for ctr in (0, 1, 12345):
+            z = oracle.splitmix64_mix((key + (ctr + 1) * gamma) % 2**64)
+            assert oracle.draw_u32(seed, ctr) == z >> 32
+    assert oracle.draw_u32(1, 0) != oracle.draw_u32(2, 0)
 
 
 def test_sample_row_dense_short_circuit():
