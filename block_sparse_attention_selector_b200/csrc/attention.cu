@@ -13,7 +13,7 @@
 //               O_g += P_g V_g; the halves are merged in the epilogue
 //   warps 8-14  loaders: TMA gathers of 32 blocks (= 128 key rows) per tile
 //               into SW128 shared-memory tiles, K and V in separate 2-stage
-//               rings, plus the tile's per-column logit bias
+//               rings, plus the tile's per-column logit bias (4-slot ring)
 //   warp 15     TMEM owner and MMA issuer (one thread):
 //              S_j = Q K_j^T  -> TMEM (two 128-column buffers)
 //              O_g += P_j[:, 64g..] V_j[64g.., :] -> TMEM (two D-column
@@ -36,10 +36,11 @@ struct AttnSmem {
     static constexpr int kKOff = kQOff + kQBytes;              // [2] stages
     static constexpr int kVOff = kKOff + 2 * kKVBytes;         // [2] stages
     static constexpr int kPOff = kVOff + 2 * kKVBytes;         // 128 x 128 bf16
-    static constexpr int kBiasOff = kPOff + 2 * kTile;         // [2][128] f32
-    static constexpr int kRedOff = kBiasOff + 2 * 128 * 4;    // [2][2][128] f32 final merge
+    static constexpr int kBiasStages = 4;
+    static constexpr int kBiasOff = kPOff + 2 * kTile;         // [4][128] f32
+    static constexpr int kRedOff = kBiasOff + kBiasStages * 128 * 4;  // [2][2][128] f32 final merge
     static constexpr int kBarOff = kRedOff + 4 * 128 * 4;
-    static constexpr int kBytes = kBarOff + 24 * 8;
+    static constexpr int kBytes = kBarOff + 32 * 8;
     // keep one CTA per SM so that the 512-column TMEM allocation never waits
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
 };
@@ -60,8 +61,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // 9 bytes/clock of such small boxes, several warps several times that.  Block
 // ids and log(pi) of the next tile are prefetched while the current tile is
 // issued.  Dense mode: one 128-row box per region from one lane.
-// K and V use separate 2-stage rings; the logit bias of the tile travels with
-// V (every loader warp arrives on v_full after writing its columns).
+// K and V use separate 2-stage rings.  The logit bias of tile t is written
+// together with K_t into slot t % 4 of its own ring (every loader warp arrives
+// on b_full after writing its columns), so the softmax of a tile never waits
+// for that tile's V.
 template <int D, bool DENSE>
 __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -85,8 +88,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     uint64_t *s_free = bars + 11;  // [2]
     uint64_t *p_full = bars + 13;  // [2] per column half
     uint64_t *p_free = bars + 15;  // [2] per column half
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
+    uint64_t *b_full = bars + 17;  // [4] logit bias of tile j in slot j % 4
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
     float *red = reinterpret_cast<float *>(sm + S::kRedOff);  // [max|sum][half][row]
 
     const int tid = threadIdx.x;
@@ -101,7 +105,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         for (int s = 0; s < 2; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
-            mbar_init(v_full + s, DENSE ? 1 : kLoadWarps);
+            mbar_init(v_full + s, 1);
             mbar_init(v_empty + s, 1);
             mbar_init(s_full + s, 1);
             mbar_init(s_free + s, kSoftmaxWarps);
@@ -110,6 +114,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             mbar_init(p_full + h, kSoftmaxWarps / 2);
             mbar_init(p_free + h, 1);
         }
+        for (int i = 0; i < S::kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kLoadWarps);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -162,168 +167,157 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         const int pbox = lw + kLoadWarps * lane;
         const int slot = pbox / R, reg = pbox % R;
         const bool has_box = pbox < 32 * R;
-        // prefetch of block id and log(pi) for tile 0
-        int b_next = -1;
-        float lp_next = 0.f;
-        if (!DENSE && has_box && slot < count) {
-            b_next = __ldg(idx_row + slot);
-            lp_next = __ldg(lp_row + slot);
-        }
-        bool ok = true;
-        for (int j = 0; j < T && ok; ++j) {
-            const int st = j & 1;
-            const int nb = min(32, count - 32 * j);
-            const int b = b_next;
-            const float lpv = lp_next;
-            if (!DENSE) {  // prefetch the next tile's entries
-                b_next = -1;
-                const int e = 32 * (j + 1) + slot;
-                if (has_box && e < count) {
-                    b_next = __ldg(idx_row + e);
-                    lp_next = __ldg(lp_row + e);
-                }
+        // this lane's plan entry (block id, log pi) in tile t; -1 past the end
+        auto entry = [&](int t, int &b, float &lp) {
+            b = -1;
+            lp = 0.f;
+            const int e = 32 * t + slot;
+            if (!DENSE && has_box && e < count) {
+                b = __ldg(idx_row + e);
+                lp = __ldg(lp_row + e);
             }
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(k_empty + st, ((j - 2) >> 1) & 1, status, abort_flag));
-                if (!ok) break;
-            }
+        };
+        // K_t and the logit bias of tile t (bias slot t % 4; a slot is
+        // rewritten only after S_{t-2} has completed, by which time the MMA
+        // order guarantees that tile t-4's softmax is done with it)
+        auto issue_k = [&](int t, int b, float lpv) -> bool {
+            const int st = t & 1;
+            if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((t - 2) >> 1) & 1,
+                                                             status, abort_flag)))
+                return false;
+            float *bias = bias_s + (t % S::kBiasStages) * 128;
             const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
             if (DENSE) {
-                if (lw == 0 && lane == 0) {
-                    mbar_arrive_expect_tx(k_full + st, S::kKVBytes);
-                    for (int r = 0; r < R; ++r)
-                        tma_load_2d(k_s + r * S::kTile, &tm_k, 64 * r, (int)(row0 + 128 * j),
-                                    k_full + st);
-                }
-            } else {
-                if (lw == 0 && lane == 0) mbar_arrive_expect_tx(k_full + st, nb * 512 * R);
-                if (b >= 0)
-                    tma_load_2d(k_s + reg * S::kTile + slot * 512, &tm_k, 64 * reg,
-                                (int)(row0 + 4 * b), k_full + st);
-            }
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(v_empty + st, ((j - 2) >> 1) & 1, status, abort_flag));
-                if (!ok) break;
-            }
-            const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
-            if (DENSE) {
                 if (lw == 0) {
-                    float4 bias;
-                    const int t0 = 128 * j + 4 * lane;
-                    bias.x = t0 < N ? 0.f : -INFINITY;
-                    bias.y = t0 + 1 < N ? 0.f : -INFINITY;
-                    bias.z = t0 + 2 < N ? 0.f : -INFINITY;
-                    bias.w = t0 + 3 < N ? 0.f : -INFINITY;
-                    reinterpret_cast<float4 *>(bias_s + st * 128)[lane] = bias;
+                    float4 bb;
+                    const int t0 = 128 * t + 4 * lane;
+                    bb.x = t0 < N ? 0.f : -INFINITY;
+                    bb.y = t0 + 1 < N ? 0.f : -INFINITY;
+                    bb.z = t0 + 2 < N ? 0.f : -INFINITY;
+                    bb.w = t0 + 3 < N ? 0.f : -INFINITY;
+                    reinterpret_cast<float4 *>(bias)[lane] = bb;
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
+                        mbar_arrive(b_full + t % S::kBiasStages);
+                        mbar_arrive_expect_tx(k_full + st, S::kKVBytes);
                         for (int r = 0; r < R; ++r)
-                            tma_load_2d(v_s + r * S::kTile, &tm_v, 64 * r, (int)(row0 + 128 * j),
-                                        v_full + st);
+                            tma_load_2d(k_s + r * S::kTile, &tm_k, 64 * r, (int)(row0 + 128 * t),
+                                        k_full + st);
                     }
                 }
             } else {
                 if (has_box && reg == 0) {  // logit bias of the block's 4 columns
-                    float4 bias = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                    float4 bb = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
                     if (b >= 0) {
                         const float sh = -lpv * kLog2e;
                         const int t0 = 4 * b;
-                        bias.x = t0 < N ? sh : -INFINITY;
-                        bias.y = t0 + 1 < N ? sh : -INFINITY;
-                        bias.z = t0 + 2 < N ? sh : -INFINITY;
-                        bias.w = t0 + 3 < N ? sh : -INFINITY;
+                        bb.x = t0 < N ? sh : -INFINITY;
+                        bb.y = t0 + 1 < N ? sh : -INFINITY;
+                        bb.z = t0 + 2 < N ? sh : -INFINITY;
+                        bb.w = t0 + 3 < N ? sh : -INFINITY;
                     }
-                    reinterpret_cast<float4 *>(bias_s + st * 128)[slot] = bias;
+                    reinterpret_cast<float4 *>(bias)[slot] = bb;
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    if (lw == 0)
-                        mbar_arrive_expect_tx(v_full + st, nb * 512 * R);
-                    else
-                        mbar_arrive(v_full + st);
+                    mbar_arrive(b_full + t % S::kBiasStages);
+                    if (lw == 0) mbar_arrive_expect_tx(k_full + st, min(32, count - 32 * t) * 512 * R);
                 }
+                if (b >= 0)
+                    tma_load_2d(k_s + reg * S::kTile + slot * 512, &tm_k, 64 * reg,
+                                (int)(row0 + 4 * b), k_full + st);
+            }
+            return true;
+        };
+        auto issue_v = [&](int t, int b) -> bool {
+            const int st = t & 1;
+            if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(v_empty + st, ((t - 2) >> 1) & 1,
+                                                             status, abort_flag)))
+                return false;
+            const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
+            if (DENSE) {
+                if (lw == 0 && lane == 0) {
+                    mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
+                    for (int r = 0; r < R; ++r)
+                        tma_load_2d(v_s + r * S::kTile, &tm_v, 64 * r, (int)(row0 + 128 * t),
+                                    v_full + st);
+                }
+            } else {
+                if (lw == 0 && lane == 0)
+                    mbar_arrive_expect_tx(v_full + st, min(32, count - 32 * t) * 512 * R);
                 if (b >= 0)
                     tma_load_2d(v_s + reg * S::kTile + slot * 512, &tm_v, 64 * reg,
                                 (int)(row0 + 4 * b), v_full + st);
             }
+            return true;
+        };
+        // Issue order K_0, then (K_{j+1}, V_j) for j = 0, 1, ...: the MMA order
+        // S_{j+2} after PV_j frees K slots one half tile ahead of V slots.
+        // Plan entries are fetched two tiles ahead.
+        int b0, b1, b2;
+        float l0, l1, l2;
+        entry(0, b0, l0);
+        entry(1, b1, l1);
+        bool ok = T > 0 ? issue_k(0, b0, l0) : true;
+        for (int j = 0; j < T && ok; ++j) {
+            entry(j + 2, b2, l2);
+            if (j + 1 < T) ok = issue_k(j + 1, b1, l1);
+            if (ok) ok = issue_v(j, b0);
+            b0 = b1;
+            l0 = l1;
+            b1 = b2;
+            l1 = l2;
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
-        // Issues S_j = Q K_j^T as soon as K_j has landed and S buffer j%2 is
-        // free, and O += P_j V_j as soon as P_j is written; whichever is ready
-        // first goes first, so neither waits behind the other's operands.
+        // One thread issues, in a fixed order, S_0, S_1 and then for every
+        // tile j: O_0 += P_j[:, 0..63] V_j[0..63, :], O_1 += P_j[:, 64..]
+        // V_j[64.., :], S_{j+2} = Q K_{j+2}^T.  Each step waits (bounded) for
+        // its operands; S_{j+2} also waits for S buffer j % 2 to be read.
         if (lane == 0 && T > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
             const uint32_t q_s = smem_u32(sm + S::kQOff);
             const uint32_t p_s = smem_u32(sm + S::kPOff);
-            bool ok = mbar_wait(q_full, 0, status, abort_flag);
-            int js = 0;            // next S tile
-            int jp[2] = {0, 0};    // next PV tile of each column half
-            long long t0 = clock64();
-            uint32_t spins = 0;
-            while (ok && (jp[0] < T || jp[1] < T)) {
-                bool progressed = false;
-                if (js < T && js < min(jp[0], jp[1]) + 2) {
-                    const int st = js & 1;
-                    if (mbar_try_wait(k_full + st, (js >> 1) & 1) &&
-                        (js < 2 || mbar_try_wait(s_free + st, ((js - 2) >> 1) & 1))) {
-                        tc_fence_after();
-                        const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
+            auto issue_s = [&](int js) -> bool {
+                const int st = js & 1;
+                if (!mbar_wait(k_full + st, (js >> 1) & 1, status, abort_flag)) return false;
+                if (js >= 2 && !mbar_wait(s_free + st, ((js - 2) >> 1) & 1, status, abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
 #pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
-                            tc_mma_f16(tmem + st * 128, sw128_desc(q_s + off, 16, 1024),
-                                       sw128_desc(k_s + off, 16, 1024), idesc_s,
-                                       ks > 0 ? 1u : 0u);
-                        }
-                        tc_commit(s_full + st);
-                        tc_commit(k_empty + st);
-                        ++js;
-                        progressed = true;
-                    }
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
+                    tc_mma_f16(tmem + st * 128, sw128_desc(q_s + off, 16, 1024),
+                               sw128_desc(k_s + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                 }
+                tc_commit(s_full + st);
+                tc_commit(k_empty + st);
+                return true;
+            };
+            auto issue_pv = [&](int j, int h) -> bool {
+                const int st = j & 1;
+                if (!mbar_wait(p_full + h, j & 1, status, abort_flag)) return false;
+                if (h == 0 && !mbar_wait(v_full + st, (j >> 1) & 1, status, abort_flag)) return false;
+                tc_fence_after();
+                // O_h += P[:, 64h .. 64h+63] V[64h .. 64h+63, :]
+                const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int j = jp[h];
-                    if (j >= js) continue;
-                    const int st = j & 1;
-                    if (!mbar_try_wait(p_full + h, j & 1) || !mbar_try_wait(v_full + st, (j >> 1) & 1))
-                        continue;
-                    tc_fence_after();
-                    // O_h += P[:, 64h .. 64h+63] V[64h .. 64h+63, :]
-                    const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t a = sw128_desc(p_s + h * S::kTile + ks * 32, 16, 1024);
-                        const uint64_t bdesc =
-                            sw128_desc(v_s + (64 * h + 16 * ks) * 128, S::kTile, 1024);
-                        tc_mma_f16(tmem_o + 128 * h, a, bdesc, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    tc_commit(p_free + h);
-                    jp[h] = j + 1;
-                    if (jp[1 - h] > j) tc_commit(v_empty + st);  // both halves of tile j issued
-                    progressed = true;
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t a = sw128_desc(p_s + h * S::kTile + ks * 32, 16, 1024);
+                    const uint64_t bdesc = sw128_desc(v_s + (64 * h + 16 * ks) * 128, S::kTile, 1024);
+                    tc_mma_f16(tmem_o + 128 * h, a, bdesc, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
                 }
-                if (progressed) {
-                    spins = 0;
-                } else {
-                    __nanosleep(32);  // leave the issue slots to the softmax warps
-                    if ((++spins & 255u) == 0) {
-                        if (*abort_flag) {
-                            ok = false;
-                        } else if (spins == 256u) {
-                            t0 = clock64();  // start of this stall
-                        } else if (clock64() - t0 > kWaitLimitCycles) {
-                            *abort_flag = 1;
-                            if (status) atomicOr(status, ABSA_DEVFLAG_TIMEOUT);
-                            ok = false;
-                        }
-                    }
-                }
+                tc_commit(p_free + h);
+                if (h == 1) tc_commit(v_empty + st);  // both halves of tile j issued
+                return true;
+            };
+            bool ok = mbar_wait(q_full, 0, status, abort_flag) && issue_s(0);
+            if (ok && T > 1) ok = issue_s(1);
+            for (int j = 0; j < T && ok; ++j) {
+                ok = issue_pv(j, 0) && issue_pv(j, 1);
+                if (ok && j + 2 < T) ok = issue_s(j + 2);
             }
         }
     } else {
@@ -354,25 +348,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free + b);
-            ok = __all_sync(0xffffffffu, mbar_wait(v_full + b, (j >> 1) & 1, status, abort_flag));
+            const int bs = j % S::kBiasStages;
+            ok = __all_sync(0xffffffffu, mbar_wait(b_full + bs, (j / S::kBiasStages) & 1, status, abort_flag));
             if (!ok) break;
-            const float *bias = bias_s + b * 128 + cb;
+            const uint32_t bias_u = smem_u32(bias_s + bs * 128 + cb);
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            const uint64_t sc2 = ((uint64_t)__float_as_uint(scale_log2) << 32) | __float_as_uint(scale_log2);
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
-                    const float4 bb = *reinterpret_cast<const float4 *>(bias + ch * 32 + i);
-                    const float x0 = __fmaf_rn(__uint_as_float(sv[ch][i]), scale_log2, bb.x);
-                    const float x1 = __fmaf_rn(__uint_as_float(sv[ch][i + 1]), scale_log2, bb.y);
-                    const float x2 = __fmaf_rn(__uint_as_float(sv[ch][i + 2]), scale_log2, bb.z);
-                    const float x3 = __fmaf_rn(__uint_as_float(sv[ch][i + 3]), scale_log2, bb.w);
-                    sv[ch][i] = __float_as_uint(x0);
-                    sv[ch][i + 1] = __float_as_uint(x1);
-                    sv[ch][i + 2] = __float_as_uint(x2);
-                    sv[ch][i + 3] = __float_as_uint(x3);
+                    uint64_t b01, b23;
+                    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
+                                 : "=l"(b01), "=l"(b23)
+                                 : "r"(bias_u + (uint32_t)(ch * 32 + i) * 4u));
+                    const uint64_t x01 = f32x2_fma(((uint64_t)sv[ch][i + 1] << 32) | sv[ch][i], sc2, b01);
+                    const uint64_t x23 = f32x2_fma(((uint64_t)sv[ch][i + 3] << 32) | sv[ch][i + 2], sc2, b23);
+                    sv[ch][i] = (uint32_t)x01;
+                    sv[ch][i + 1] = (uint32_t)(x01 >> 32);
+                    sv[ch][i + 2] = (uint32_t)x23;
+                    sv[ch][i + 3] = (uint32_t)(x23 >> 32);
                     const int a = (i >> 2) & 3;
-                    mx4[a] = fmaxf(mx4[a], fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+                    mx4[a] = fmaxf(mx4[a], fmaxf(fmaxf(__uint_as_float(sv[ch][i]), __uint_as_float(sv[ch][i + 1])),
+                                                 fmaxf(__uint_as_float(sv[ch][i + 2]), __uint_as_float(sv[ch][i + 3]))));
                 }
             const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             // lazy max: keep the reference unless the tile exceeds it by 2^8;
@@ -387,18 +385,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 if (!ok) break;
             }
             const float moff = m_ref == -INFINITY ? 0.f : -m_ref;
-            float acc8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc8[i] = 0.f;
+            const uint64_t moff2 = ((uint64_t)__float_as_uint(moff) << 32) | __float_as_uint(moff);
+            uint64_t acc2[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {  // 8 columns = one 16-byte chunk
                     float p[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        p[e] = ex2(__uint_as_float(sv[ch][g * 8 + e]) + moff);
-                        acc8[e] += p[e];
+                    for (int e = 0; e < 8; e += 2) {
+                        const uint64_t y2 = f32x2_add(((uint64_t)sv[ch][g * 8 + e + 1] << 32) | sv[ch][g * 8 + e], moff2);
+                        p[e] = ex2(__uint_as_float((uint32_t)y2));
+                        p[e + 1] = ex2(__uint_as_float((uint32_t)(y2 >> 32)));
+                        acc2[e >> 1] = f32x2_add(acc2[e >> 1], ((uint64_t)__float_as_uint(p[e + 1]) << 32) | __float_as_uint(p[e]));
                     }
                     const uint32_t dst = p_s + sw128_offset(r, ch * 4 + g);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
@@ -422,8 +421,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 }
                 tmem_wait_st();
             }
-            lsum += ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
-                    ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+            {
+                const uint64_t a01 = f32x2_add(acc2[0], acc2[1]), a23 = f32x2_add(acc2[2], acc2[3]);
+                const uint64_t a = f32x2_add(a01, a23);
+                lsum += __uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)(a >> 32));
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();

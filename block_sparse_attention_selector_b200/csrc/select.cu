@@ -72,17 +72,6 @@ __global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__r
 //                         conflicts: a warp reads 32 consecutive columns of one
 //                         row), mu = sum / count (IEEE division); an empty
 //                         cluster keeps mu.
-__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
 template <int D>
 struct KmeansSmem {
     static constexpr int kRow = D + 2;                  // bf16 row pitch: 4*(D/2+1) bytes, so
@@ -101,7 +90,6 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     uint8_t *__restrict__ assign_out) {
     using S = KmeansSmem<D>;
     constexpr int NC = 8;
-    constexpr int CH = D / 8;  // 16-byte chunks per row
     extern __shared__ __align__(16) uint8_t kms[];
     __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(kms + S::kX);
     float *mut = reinterpret_cast<float *>(kms + S::kMu);
