@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads (profiling captures); 0 = all 40")
     ap.add_argument("--dense-reps", type=int, default=3)
+    ap.add_argument("--sweep", action="store_true",
+                    help="density sweep and 16-step plan-reuse schedule (JSON lines; no main line)")
     return ap.parse_args()
 
 
@@ -380,10 +382,105 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ sweep
+
+SWEEP_BUDGETS = (82, 164, 410, 819, 2048, 8190)  # round-half-up of 1, 2, 5, 10, 25, 100% of 8190
+
+
+def run_sweep(args):
+    """Density sweep (budgets above, 8 sampling seeds, one plan reused for 4 calls) and the
+    16-step plan-reuse schedule (a new plan every 4th step, q/k drifting by 0.05 N(0,1) per
+    step), each against our dense kernel on the same inputs.  Prints one JSON line per budget
+    and one for the schedule."""
+    import torch
+
+    import block_sparse_attention_selector_b200 as absa
+    from block_sparse_attention_selector_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    w = workload(args.heads)
+    q_bits, k_bits, v_bits = synthetic.layer_qkv_bits(w)
+
+    def to_dev(b):
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q, k, v = to_dev(q_bits), to_dev(k_bits), to_dev(v_bits)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        out = fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return out, e0.elapsed_time(e1)
+
+    def rel_l2(a, b):
+        a, b = a.float(), b.float()
+        return float((a - b).norm() / b.norm())
+
+    p0 = absa.params_for(w)
+    for _ in range(2):
+        o_dense, dense_ms = timed(lambda: absa.dense_reference(p0, q, k, v))
+    dense_rms = float(o_dense.float().pow(2).mean().sqrt())
+    v_rms = float(v.float().pow(2).mean().sqrt())
+    for budget in SWEEP_BUDGETS:
+        sel, att, rel, blocks = [], [], [], []
+        for seed in range(8):
+            p = absa.params_for(w, seed=seed, budget=budget)
+            (plan, _, _), t_sel = timed(lambda: absa.select_plan(p, q, k))
+            plan.check()
+            for _ in range(4):  # one plan, four attention calls
+                o, t_att = timed(lambda: absa.sparse_attention(p, q, k, v, plan))
+                att.append(t_att)
+            sel.append(t_sel)
+            rel.append(rel_l2(o, o_dense))
+            blocks.append(float(plan.counts.float().mean()))
+        line = {"kind": "density_sweep", "workload": w.name, "budget_blocks": budget,
+                "density": budget / w.nkb, "mean_blocks_per_row": float(np.mean(blocks)),
+                "select_plan_ms": float(np.median(sel)), "attention_ms": float(np.median(att)),
+                "ms_per_call_plan_reused_4x": float(np.median(sel)) / 4 + float(np.median(att)),
+                "dense_ms": dense_ms, "rel_l2_vs_dense_mean_8_seeds": float(np.mean(rel)),
+                "rel_l2_vs_dense_std_8_seeds": float(np.std(rel)),
+                # v is N(0,1) noise, so the dense output (an average of many v rows) is small
+                # next to v; these two set the scale of the relative error above
+                "dense_output_rms": dense_rms, "v_rms": v_rms}
+        print(json.dumps(line), flush=True)
+
+    # 16-step schedule at the layer's budget; the per-step noise is drawn on the GPU from a
+    # generator seeded with (workload seed, step)
+    p = absa.params_for(w, seed=1)
+    qf, kf = q.float(), k.float()
+    gen = torch.Generator(device=dev)
+    steps, plan_ms, att_ms, rels = 16, [], [], []
+    for step in range(steps):
+        if step > 0:
+            gen.manual_seed(1000 * (w.seed + 1) + step)
+            qf += 0.05 * torch.randn(qf.shape, generator=gen, device=dev)
+            kf += 0.05 * torch.randn(kf.shape, generator=gen, device=dev)
+            q, k = qf.to(torch.bfloat16), kf.to(torch.bfloat16)
+        if step % 4 == 0:
+            (plan, _, _), t = timed(lambda: absa.select_plan(p, q, k))
+            plan.check()
+            plan_ms.append(t)
+        o, t = timed(lambda: absa.sparse_attention(p, q, k, v, plan))
+        att_ms.append(t)
+        rels.append(rel_l2(o, absa.dense_reference(p, q, k, v)))
+    line = {"kind": "plan_reuse_schedule", "workload": w.name, "steps": steps, "plan_every": 4,
+            "drift_sigma_per_step": 0.05, "ms_per_step": (sum(plan_ms) + sum(att_ms)) / steps,
+            "select_plan_ms": plan_ms, "attention_ms_mean": float(np.mean(att_ms)),
+            "rel_l2_vs_dense_per_step": rels}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 

@@ -22,6 +22,22 @@ __device__ __forceinline__ uint64_t quantise_score(float s) {
 
 constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;  // SplitMix64 increment
 
+// Upper 32 bits of the SplitMix64 output function of z.  Only the high word
+// of the second product and of the last xor-shift is formed: with
+// z = hi 2^32 + lo, the high word of z * c mod 2^64 is
+// hi32(lo * c_lo) + lo * c_hi + hi * c_lo (mod 2^32), and the high word of
+// z ^ (z >> 31) is hi ^ (hi >> 31).
+__device__ __forceinline__ uint32_t splitmix64_hi32(uint64_t z) {
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z ^= z >> 27;
+    const uint32_t lo = (uint32_t)z, hi = (uint32_t)(z >> 32);
+    const uint32_t h = __umulhi(lo, 0x133111EBu) + lo * 0x94D049BBu + hi * 0x133111EBu;
+    return h ^ (h >> 31);
+}
+
+// Candidate list for the capping rounds after the first (see the kernel).
+constexpr int kCandMax = 2048;
+
 // u * R < rq * 2^32 exactly (u < 2^32, R < 2^48, rq < 2^48): with
 // R = Rh 2^32 + Rl, u R = (u Rh + hi32(u Rl)) 2^32 + lo32(u Rl), so the
 // comparison reduces to u Rh + hi32(u Rl) < rq.
@@ -58,8 +74,16 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
 // One CTA per plan row (b,h,qb).  Key blocks are handled in groups of 32 (one
 // per lane); warp w owns a contiguous run of groups, so the taken blocks of
 // warp w all precede those of warp w+1 and one scan of the 8 warp counts
-// places every entry.  Shared memory: q_j - 1 as u32 per block, plus one
-// capped word and one taken word (ballots) per group.
+// places every entry.  Shared memory: q_j - 1 as u32 per block, one capped
+// word and one taken word (ballots) per group, and the candidate list.
+//
+// Capping: the first round (r = n, R = sum q) runs over every block and also
+// lists the blocks with 2 n q_j >= R_total, i.e. q_j at least half of the
+// first threshold R/r.  The threshold only decreases from round to round, and
+// while it stays at or above that half every block a later round caps is on
+// the list, so warp 0 runs those rounds over the list alone.  If the list
+// overflows or the threshold falls below the half, the remaining rounds scan
+// every block.  Either way the rounds are exactly those of the definition.
 __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
@@ -69,9 +93,13 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     uint32_t *qm1 = samp_smem;                      // [ngroups*32]
     uint32_t *capw = samp_smem + ngroups * 32;      // [ngroups]
     uint32_t *takew = capw + ngroups;               // [ngroups]
+    uint32_t *cand = takew + ngroups;               // [kCandMax]
     __shared__ uint64_t red_a[kSampleWarps];
     __shared__ int red_b[kSampleWarps];
     __shared__ int warp_cnt[kSampleWarps];
+    __shared__ int n_cand;
+    __shared__ uint64_t fin_R;
+    __shared__ int fin_capped, fin_full;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = blockIdx.x;
@@ -98,58 +126,146 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const int g1 = min(ngroups, g0 + per_warp);
 
     // quantise once; R = sum of all q_j
+    if (tid == 0) n_cand = 0;
     uint64_t R = 0;
     int dummy = 0;
-    for (int g = g0; g < g1; ++g) {
-        const int j = g * 32 + lane;
-        uint64_t qj = 0;
-        if (j < nkb) {
-            qj = quantise_score(__ldg(srow + j));
-            qm1[j] = (uint32_t)(qj - 1);
+    for (int g = g0; g < g1; g += 8) {  // 8 loads in flight per lane
+        float sv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int j = (g + u) * 32 + lane;
+            sv[u] = (g + u < g1 && j < nkb) ? __ldg(srow + j) : 0.f;
         }
-        R += qj;
-        if (lane == 0) capw[g] = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int j = (g + u) * 32 + lane;
+            if (g + u < g1 && j < nkb) {
+                const uint64_t qj = quantise_score(sv[u]);
+                qm1[j] = (uint32_t)(qj - 1);
+                R += qj;
+            }
+        }
     }
     block_sum2(R, dummy, red_a, red_b);
+    const uint64_t R0 = R;
+    const uint64_t nn = (uint64_t)n;
 
-    // capping fixed point: mark with (r, R), then the rest's sum is the next R
-    int n_capped = 0;
-    uint64_t r = (uint64_t)n;
-    uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
-    for (;;) {
-        uint64_t rest = 0;
-        int grew = 0;
-        for (int g = g0; g < g1; ++g) {
-            const int j = g * 32 + lane;
-            const uint32_t word = capw[g];
-            bool newcap = false;
-            if (j < nkb && !((word >> lane) & 1u)) {
-                const uint32_t q1 = qm1[j];
-                if ((uint64_t)r32 * q1 + r32 >= R)  // r * q_j
-                    newcap = true;
-                else
-                    rest += (uint64_t)q1 + 1;
-            }
-            const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
-            if (nb) {
-                if (lane == 0) capw[g] = word | nb;
-                grew += lane == 0 ? __popc(nb) : 0;
+    // round 1 over every block (r = n), listing the candidates for later rounds
+    const uint32_t below = (1u << lane) - 1u;
+    uint64_t capsum = 0;
+    int capcnt = 0;
+    for (int g = g0; g < g1; ++g) {
+        const int j = g * 32 + lane;
+        bool newcap = false, is_cand = false;
+        if (j < nkb) {
+            const uint64_t q = (uint64_t)qm1[j] + 1;
+            if (nn * q >= R0) {
+                newcap = true;
+                capsum += q;
+                ++capcnt;
+            } else if (2 * nn * q >= R0) {
+                is_cand = true;
             }
         }
-        block_sum2(rest, grew, red_a, red_b);
-        if (grew == 0) break;
-        n_capped += grew;
-        r = (uint64_t)(n - n_capped);
-        r32 = (uint32_t)r;
-        R = rest;
+        const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
+        if (lane == 0) capw[g] = nb;
+        const uint32_t cb = __ballot_sync(0xffffffffu, is_cand);
+        if (cb) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&n_cand, __popc(cb));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int p = base + __popc(cb & below);
+            if (is_cand && p < kCandMax) cand[p] = (uint32_t)j;
+        }
     }
+    block_sum2(capsum, capcnt, red_a, red_b);
+    int n_capped = capcnt;
+    uint64_t r = nn - (uint64_t)n_capped;
+    R = R0 - capsum;
+
+    // later rounds over the candidate list (warp 0)
+    if (warp == 0) {
+        const int nc = n_cand;
+        bool full = nc > kCandMax;
+        bool grew = capcnt > 0;
+        while (grew && !full) {
+            // the list holds every block this round can cap iff R / r >= R0 / (2 n)
+            if ((unsigned __int128)(2 * nn) * R < (unsigned __int128)r * R0) {
+                full = true;
+                break;
+            }
+            uint64_t s = 0;
+            int c = 0;
+            for (int i = lane; i < nc; i += 32) {
+                const uint32_t j = cand[i];
+                if (!((capw[j >> 5] >> (j & 31)) & 1u)) {
+                    const uint64_t q = (uint64_t)qm1[j] + 1;
+                    if (r * q >= R) {
+                        s += q;
+                        ++c;
+                        atomicOr(&capw[j >> 5], 1u << (j & 31));
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, o);
+                c += __shfl_xor_sync(0xffffffffu, c, o);
+            }
+            grew = c > 0;
+            n_capped += c;
+            r -= (uint64_t)c;
+            R -= s;
+            __syncwarp();  // this round's marks are visible to the next round's reads
+        }
+        if (lane == 0) {
+            fin_R = R;
+            fin_capped = n_capped;
+            fin_full = full ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    R = fin_R;
+    n_capped = fin_capped;
+    r = nn - (uint64_t)n_capped;
+    if (fin_full) {
+        // remaining rounds scan every block (the state so far is exact)
+        for (;;) {
+            uint64_t newsum = 0;
+            int grew = 0;
+            for (int g = g0; g < g1; ++g) {
+                const int j = g * 32 + lane;
+                const uint32_t word = capw[g];
+                bool newcap = false;
+                if (j < nkb && !((word >> lane) & 1u)) {
+                    const uint64_t q = (uint64_t)qm1[j] + 1;
+                    if (r * q >= R) {
+                        newcap = true;
+                        newsum += q;
+                    }
+                }
+                const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
+                if (nb) {
+                    if (lane == 0) capw[g] = word | nb;
+                    grew += lane == 0 ? __popc(nb) : 0;
+                }
+            }
+            block_sum2(newsum, grew, red_a, red_b);
+            if (grew == 0) break;
+            n_capped += grew;
+            r = nn - (uint64_t)n_capped;
+            R -= newsum;
+        }
+    }
+    const uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
 
     // Poisson draws: one taken word per group; SplitMix64 state of block j is
     // base + j * gamma with base = mix(seed) + (row * NKB + 1) * gamma
     const uint64_t base = splitmix64_mix(seed) + ((uint64_t)row * (uint64_t)nkb + 1) * kGamma;
     const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
     int taken = 0;
-    for (int g = g0; g < g1; ++g) {
+    uint64_t state = base + (uint64_t)(g0 * 32 + lane) * kGamma;  // state of block j
+    for (int g = g0; g < g1; ++g, state += 32 * kGamma) {
         const int j = g * 32 + lane;
         bool take = false;
         if (j < nkb) {
@@ -157,8 +273,7 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
                 take = true;
             } else {
                 const uint64_t rq = (uint64_t)r32 * qm1[j] + r32;
-                const uint32_t u = (uint32_t)(splitmix64_mix(base + (uint64_t)j * kGamma) >> 32);
-                take = draw_taken(u, Rh, Rl, rq);
+                take = draw_taken(splitmix64_hi32(state), Rh, Rl, rq);
             }
         }
         const uint32_t tw = __ballot_sync(0xffffffffu, take);
@@ -174,13 +289,18 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         pos += w < warp ? c : 0;
         total += c;
     }
-    // ascending compaction of this warp's run (block ids only)
-    const uint32_t below = (1u << lane) - 1u;
+    // ascending compaction of this warp's run (block ids only); the ids are
+    // also kept in shared memory (the candidate list is no longer needed)
+    // for the logarithm pass when they fit
+    const bool ids_in_smem = min(total, cap) <= kCandMax;
     for (int g = g0; g < g1 && pos < cap; ++g) {
         const uint32_t tw = takew[g];
         if ((tw >> lane) & 1u) {
             const int p = pos + __popc(tw & below);
-            if (p < cap) idx_row[p] = g * 32 + lane;
+            if (p < cap) {
+                idx_row[p] = g * 32 + lane;
+                if (ids_in_smem) cand[p] = (uint32_t)(g * 32 + lane);
+            }
         }
         pos += __popc(tw);
     }
@@ -189,7 +309,7 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     // logarithm would otherwise run for a whole warp per taken lane)
     const int written = min(total, cap);
     for (int p = tid; p < written; p += kSampleThreads) {
-        const int j = idx_row[p];
+        const int j = ids_in_smem ? (int)cand[p] : idx_row[p];
         float lp = 0.f;
         if (!((capw[j >> 5] >> (j & 31)) & 1u))
             lp = (float)log((double)((uint64_t)r32 * qm1[j] + r32) / (double)R);
@@ -207,7 +327,7 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
                           int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
                           uint64_t *r_R, int32_t *status, cudaStream_t stream) {
     const int ngroups = (nkb + 31) / 32;
-    const int smem = (ngroups * 32 + 2 * ngroups) * 4;
+    const int smem = (ngroups * 32 + 2 * ngroups + kCandMax) * 4;
     cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
