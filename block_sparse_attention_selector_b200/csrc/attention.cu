@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     uint64_t *b_full = bars + 17;  // [4] logit bias of tile j in slot j % 4
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
+    int *bad_flag = reinterpret_cast<int *>(bars + 23);  // a plan entry out of range
     float *red = reinterpret_cast<float *>(sm + S::kRedOff);  // [max|sum][half][row]
 
     const int tid = threadIdx.x;
@@ -116,33 +117,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         }
         for (int i = 0; i < S::kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kLoadWarps);
         *abort_flag = 0;
+        *bad_flag = 0;
         mbar_fence_init();
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
-    // Rows of a partial tile that no box overwrites must hold finite values
-    // (P = 0 there, and 0 * NaN would poison O): clear the K/V rings once.
-    for (int i = tid; i < 4 * S::kKVBytes / 16; i += kAttnThreads)
-        reinterpret_cast<uint4 *>(sm + S::kKOff)[i] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
 
-    // number of plan entries; reject a malformed plan row (it is written as zeros)
+    // Number of plan entries: a count outside [0, cap] rejects the row (it is
+    // written as zeros).  Entries outside [0, NKB) are caught by the loaders,
+    // which read them anyway: such an entry loads block 0 instead and the row
+    // is written as zeros at the end.
     int count;
     if (DENSE) {
         count = nkb;
     } else {
         count = __ldg(counts + row);
-        bool bad = count < 0 || count > cap;
-        if (!bad)
-            for (int i = tid; i < count; i += kAttnThreads) {
-                const int b = __ldg(kv_index + row * cap + i);
-                bad |= (b < 0) | (b >= nkb);
-            }
-        if (__syncthreads_or(bad)) {
+        if (count < 0 || count > cap) {
             if (tid == 0) atomicOr(status, ABSA_DEVFLAG_BAD_PLAN);
             count = 0;
         }
     }
     const int T = (count + 31) / 32;
+    // Rows of a partial tile that no box overwrites must hold finite values
+    // (P = 0 there, and 0 * NaN would poison O).  After its first use a ring
+    // stage holds finite stale rows, so only a row whose first two tiles are
+    // not both full needs the rings cleared (dense tiles past N are zero-filled
+    // by the TMA unit).
+    if (!DENSE && count < 64)
+        for (int i = tid; i < 4 * S::kKVBytes / 16; i += kAttnThreads)
+            reinterpret_cast<uint4 *>(sm + S::kKOff)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
 
     tc_fence_before();
     __syncthreads();
@@ -177,11 +180,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 lp = __ldg(lp_row + e);
             }
         };
+        // An entry of tile t present in the plan but outside [0, NKB) loads
+        // block 0 instead and marks the row (checked where the entry is used,
+        // a tile after its load, so the check adds no load latency).
+        auto checked = [&](int t, int b) -> int {
+            if (!DENSE && has_box && 32 * t + slot < count && (b < 0 || b >= nkb)) {
+                atomicOr(bad_flag, 1);
+                return 0;
+            }
+            return b;
+        };
         // K_t and the logit bias of tile t (bias slot t % 4; a slot is
         // rewritten only after S_{t-2} has completed, by which time the MMA
         // order guarantees that tile t-4's softmax is done with it)
         auto issue_k = [&](int t, int b, float lpv) -> bool {
             const int st = t & 1;
+            b = checked(t, b);
             if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((t - 2) >> 1) & 1,
                                                              status, abort_flag)))
                 return false;
@@ -231,6 +245,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         };
         auto issue_v = [&](int t, int b) -> bool {
             const int st = t & 1;
+            b = checked(t, b);
             if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(v_empty + st, ((t - 2) >> 1) & 1,
                                                              status, abort_flag)))
                 return false;
@@ -443,13 +458,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
         const float ltot = red[256 + r] * a0 + red[384 + r] * a1;
         constexpr int OC = D / 2;
-        __nv_bfloat16 *orow = o + (bh * N + (int64_t)qb * 128 + r) * D + half * OC;
-        if (T > 0 && ok) {
+        // The output tile goes through shared memory (the K ring, idle by now:
+        // every K tile has been consumed) so that the global stores are
+        // coalesced: rows of D bf16 with a 16-byte pad against bank conflicts.
+        constexpr int kStageRow = D + 8;
+        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + S::kKOff);
+        // a plan entry out of range (seen by the loaders before their last
+        // arrival on b_full, which every softmax warp has waited for)
+        const bool bad_row = !DENSE && T > 0 && *reinterpret_cast<volatile int *>(bad_flag) != 0;
+        if (T > 0 && ok && !bad_row) {
             ok = __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, status, abort_flag) &&
                                              mbar_wait(p_free + 1, (T - 1) & 1, status, abort_flag));
         }
-        if (T > 0 && ok) {
+        const bool write = T > 0 && ok && !bad_row;
+        if (write) {
             tc_fence_after();
+            fence_proxy_async_smem();  // generic writes after the ring's async-proxy use
             const float inv = 1.f / ltot;
             const float c0 = a0 * inv, c1 = a1 * inv;
 #pragma unroll
@@ -458,27 +482,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 tmem_ld32(tmem_o + lane_base + half * OC + ch * 32, o0);
                 tmem_ld32(tmem_o + 128 + lane_base + half * OC + ch * 32, o1);
                 tmem_wait_ld();
-                if (r < m) {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        float f[8];
+                for (int g = 0; g < 4; ++g) {
+                    float f[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            f[e] = __uint_as_float(o0[8 * g + e]) * c0 +
-                                   __uint_as_float(o1[8 * g + e]) * c1;
-                        uint4 u;
-                        u.x = pack_bf16x2(f[0], f[1]);
-                        u.y = pack_bf16x2(f[2], f[3]);
-                        u.z = pack_bf16x2(f[4], f[5]);
-                        u.w = pack_bf16x2(f[6], f[7]);
-                        *reinterpret_cast<uint4 *>(orow + ch * 32 + 8 * g) = u;
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        f[e] = __uint_as_float(o0[8 * g + e]) * c0 +
+                               __uint_as_float(o1[8 * g + e]) * c1;
+                    uint4 u;
+                    u.x = pack_bf16x2(f[0], f[1]);
+                    u.y = pack_bf16x2(f[2], f[3]);
+                    u.z = pack_bf16x2(f[4], f[5]);
+                    u.w = pack_bf16x2(f[6], f[7]);
+                    *reinterpret_cast<uint4 *>(stage + r * kStageRow + half * OC + ch * 32 + 8 * g) = u;
                 }
             }
-        } else if (T == 0 && r < m) {
-            const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int c = 0; c < OC / 8; ++c) *reinterpret_cast<uint4 *>(orow + c * 8) = z;
+        }
+        if (bad_row && tid == 0) atomicOr(status, ABSA_DEVFLAG_BAD_PLAN);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        // coalesced rows: consecutive threads write consecutive 16-byte chunks
+        __nv_bfloat16 *obase = o + (bh * N + (int64_t)qb * 128) * D;
+        for (int c = tid; c < m * (D / 8); c += 32 * kSoftmaxWarps) {
+            const int rr = c / (D / 8), c8 = c % (D / 8);
+            const uint4 u = write ? *reinterpret_cast<const uint4 *>(stage + rr * kStageRow + 8 * c8)
+                                  : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(obase + (int64_t)rr * D + 8 * c8) = u;
         }
     }
     tc_fence_before();
