@@ -12,8 +12,9 @@
 //               (thread = TMEM lane = query row) with its own accumulator
 //               O_g += P_g V_g; the halves are merged in the epilogue
 //   warps 8-14  loaders: TMA gathers of 32 blocks (= 128 key rows) per tile
-//               into SW128 shared-memory tiles, K and V in separate 2-stage
-//               rings, plus the tile's per-column logit bias (4-slot ring)
+//               into SW128 shared-memory tiles; warps 8-10 fill the 2-stage
+//               K ring and the tile's per-column logit bias (4-slot ring),
+//               warps 11-14 the 2-stage V ring, each group at its own pace
 //   warp 15     TMEM owner and MMA issuer (one thread):
 //              S_j = Q K_j^T  -> TMEM (two 128-column buffers)
 //              O_g += P_j[:, 64g..] V_j[64g.., :] -> TMEM (two D-column
@@ -48,6 +49,7 @@ struct AttnSmem {
 constexpr int kSoftmaxWarps = 8;              // two warpgroups, 64 columns each
 constexpr int kLoadWarp = kSoftmaxWarps;      // first loader warp
 constexpr int kLoadWarps = 7;                 // warps issuing TMA boxes
+constexpr int kKLoadWarps = 3;                // of which the K group (the rest load V)
 constexpr int kMmaWarp = kLoadWarp + kLoadWarps;   // 15
 constexpr int kAttnThreads = 32 * (kMmaWarp + 1);  // 512
 constexpr float kLog2e = 1.4426950408889634f;
@@ -56,11 +58,12 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Loaders.  Sparse mode: a tile's 32 blocks x (d/64) column regions are 4-row
 // TMA boxes (512 bytes each) placed at rows 4i..4i+3 of the SW128 tile; the
 // box swizzle follows the shared-memory address, so a box in the upper half
-// of a 1024-byte atom lands in that half's chunk order.  The boxes are spread
-// over 7 warps (box p goes to warp p % 7): a single warp sustains only about
-// 9 bytes/clock of such small boxes, several warps several times that.  Block
-// ids and log(pi) of the next tile are prefetched while the current tile is
-// issued.  Dense mode: one 128-row box per region from one lane.
+// of a 1024-byte atom lands in that half's chunk order.  A group's boxes are
+// spread over its warps (box p goes to warp p % n): a single warp sustains
+// only about 9 bytes/clock of such small boxes, several warps several times
+// that.  Block ids and log(pi) of the next tile are prefetched while the
+// current tile is issued.  Dense mode: one 128-row box per region from one
+// lane.
 // K and V use separate 2-stage rings.  The logit bias of tile t is written
 // together with K_t into slot t % 4 of its own ring (every loader warp arrives
 // on b_full after writing its columns), so the softmax of a tile never waits
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             mbar_init(p_full + h, kSoftmaxWarps / 2);
             mbar_init(p_free + h, 1);
         }
-        for (int i = 0; i < S::kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kLoadWarps);
+        for (int i = 0; i < S::kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kKLoadWarps);
         *abort_flag = 0;
         *bad_flag = 0;
         mbar_fence_init();
@@ -156,6 +159,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     if (warp >= kLoadWarp && warp < kLoadWarp + kLoadWarps) {
         // ------------------------------------------------------------ loaders
         const int lw = warp - kLoadWarp;      // 0..6
+        const bool kside = lw < kKLoadWarps;  // K group (K tiles and bias) or V group
+        const int gw = kside ? lw : lw - kKLoadWarps;              // warp within the group
+        const int gn = kside ? kKLoadWarps : kLoadWarps - kKLoadWarps;  // warps in the group
         const int64_t row0 = bh * N;          // first token row of this head
         if (lw == 0 && lane == 0 && T > 0) {
             mbar_arrive_expect_tx(q_full, S::kQBytes);
@@ -165,9 +171,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         }
         const int32_t *idx_row = DENSE ? nullptr : kv_index + row * cap;
         const float *lp_row = DENSE ? nullptr : log_pi + row * cap;
-        // box p = lw + 7 * lane of a tile: block slot p / R, region p % R
+        // box p = gw + gn * lane of a tile: block slot p / R, region p % R
         constexpr int R = S::kRegions;
-        const int pbox = lw + kLoadWarps * lane;
+        const int pbox = gw + gn * lane;
         const int slot = pbox / R, reg = pbox % R;
         const bool has_box = pbox < 32 * R;
         // this lane's plan entry (block id, log pi) in tile t; -1 past the end
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(b_full + t % S::kBiasStages);
-                    if (lw == 0) mbar_arrive_expect_tx(k_full + st, min(32, count - 32 * t) * 512 * R);
+                    if (gw == 0) mbar_arrive_expect_tx(k_full + st, min(32, count - 32 * t) * 512 * R);
                 }
                 if (b >= 0)
                     tma_load_2d(k_s + reg * S::kTile + slot * 512, &tm_k, 64 * reg,
@@ -251,14 +257,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 return false;
             const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
             if (DENSE) {
-                if (lw == 0 && lane == 0) {
+                if (gw == 0 && lane == 0) {
                     mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
                     for (int r = 0; r < R; ++r)
                         tma_load_2d(v_s + r * S::kTile, &tm_v, 64 * r, (int)(row0 + 128 * t),
                                     v_full + st);
                 }
             } else {
-                if (lw == 0 && lane == 0)
+                if (gw == 0 && lane == 0)
                     mbar_arrive_expect_tx(v_full + st, min(32, count - 32 * t) * 512 * R);
                 if (b >= 0)
                     tma_load_2d(v_s + reg * S::kTile + slot * 512, &tm_v, 64 * reg,
@@ -266,22 +272,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             }
             return true;
         };
-        // Issue order K_0, then (K_{j+1}, V_j) for j = 0, 1, ...: the MMA order
-        // S_{j+2} after PV_j frees K slots one half tile ahead of V slots.
-        // Plan entries are fetched two tiles ahead.
-        int b0, b1, b2;
-        float l0, l1, l2;
+        // Each group walks the tiles at its own pace (the K group also writes
+        // the bias); plan entries are fetched one tile ahead.
+        int b0, b1;
+        float l0, l1;
         entry(0, b0, l0);
-        entry(1, b1, l1);
-        bool ok = T > 0 ? issue_k(0, b0, l0) : true;
-        for (int j = 0; j < T && ok; ++j) {
-            entry(j + 2, b2, l2);
-            if (j + 1 < T) ok = issue_k(j + 1, b1, l1);
-            if (ok) ok = issue_v(j, b0);
+        bool ok = true;
+        for (int t = 0; t < T && ok; ++t) {
+            entry(t + 1, b1, l1);
+            ok = kside ? issue_k(t, b0, l0) : issue_v(t, b0);
             b0 = b1;
             l0 = l1;
-            b1 = b2;
-            l1 = l2;
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
