@@ -197,12 +197,14 @@ class ClockSampler:
 # ------------------------------------------------------------------ GPU arm
 
 def measured_peaks():
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, HBM GB/s, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return d.get("bf16_tflops", 1590.0), d.get("hbm_gbs", 6650.0), "measured"
-    return 1590.0, 6650.0, "fallback"
+        burst = d.get("bf16_tflops", 1590.0)
+        return burst, d.get("bf16_tflops_sustained", burst), d.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
 
 
 def recorded_traffic(kernel_src):
@@ -338,7 +340,14 @@ def run_ours(args):
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_ms = float(te.item()) / (max(1, len(e2e)) * world) if e2e else None
 
-    peak_tf, hbm_gbs, peak_src = measured_peaks()
+    burst_tf, sustained_tf, hbm_gbs, peak_src = measured_peaks()
+    clk = clocks.summary()
+    # The timed region is a loop of K steps; once it runs long enough for the
+    # power cap to act (or the sampler saw it act) the matching denominator is
+    # the sustained GEMM figure, otherwise the burst one.
+    long_loop = float(tot.sum()) >= 500.0 or "sw_power_cap" in clk.get("reasons", [])
+    peak_tf = sustained_tf if long_loop else burst_tf
+    peak_kind = "sustained" if long_loop else "burst"
     att_ms = float(att.mean())
     achieved_tf = attn_flops / (att_ms * 1e-3) / 1e12
     sel_bytes = 2 * q.numel() * 2  # algorithmic: read q and k once
@@ -363,14 +372,17 @@ def run_ours(args):
             }),
             "roofline": {"bound": "tensor", "kernel": "absa_attention_kernel<128,sparse>",
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": achieved_tf / peak_tf, "peak_source": f"{peak_src} bf16 (burst)",
+                         "frac": achieved_tf / peak_tf,
+                         "peak_source": f"{peak_src} bf16 ({peak_kind}; timed region "
+                                        f"{float(tot.sum()):.0f} ms)",
+                         "frac_of_burst_peak": achieved_tf / burst_tf,
                          "traffic": recorded_traffic(os.path.join(
                              ROOT, "block_sparse_attention_selector_b200", "csrc", "attention.cu")),
                          "algorithmic_flops_per_launch": attn_flops},
             "e2e": {"value": e2e_ms, "unit": "ms",
                     "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2},
             "gpu_launches": 5 * K,
-            "clocks": clocks.summary(),
+            "clocks": clk,
         }
     if world > 1:
         dist.barrier()
