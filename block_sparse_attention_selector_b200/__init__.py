@@ -12,15 +12,16 @@ import math
 from . import _abi
 from ._abi import (AbsaError, absa_check_params, absa_dense_reference, absa_params, absa_plan,
                    absa_plan_capacity, absa_plan_check, absa_sample_plan, absa_select_plan,
-                   absa_select_scores, absa_sparse_attention, absa_workspace_bytes)
+                   absa_select_scores, absa_sparse_attention, absa_step_host,
+                   absa_workspace_bytes)
 from .synthetic import Workload
 
 __all__ = [
     "AbsaError", "Plan", "Workload", "absa_check_params", "absa_dense_reference", "absa_params",
     "absa_plan", "absa_plan_capacity", "absa_plan_check", "absa_sample_plan", "absa_select_plan",
-    "absa_select_scores", "absa_sparse_attention", "absa_workspace_bytes", "dense_reference",
-    "make_params", "sample_plan", "select_plan", "select_scores", "sparse_attention",
-    "workspace", "version",
+    "absa_select_scores", "absa_sparse_attention", "absa_step_host", "absa_workspace_bytes",
+    "dense_reference", "make_params", "sample_plan", "select_plan", "select_scores",
+    "sparse_attention", "step_host", "workspace", "version",
 ]
 
 
@@ -158,3 +159,26 @@ def dense_reference(p, q, k, v, out=None, status=None, stream=None):
     _abi.check(absa_dense_reference(p, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(status),
                                     _stream_handle(stream)), "absa_dense_reference")
     return out
+
+
+def step_host(p, q_host, k_host, v_host, o_host, q, k, v, o, plan, scores, ws, heads_per_run=4,
+              stream=None, copy_in_stream=None, copy_out_stream=None):
+    """absa_step_host: the whole step on host bf16 tensors, pipelined over runs of heads.
+
+    q_host, k_host, v_host, o_host are contiguous bf16 CPU tensors [B,H,N,d] (pin them for the
+    copies to overlap the compute); q, k, v, o, plan, scores, ws are the device buffers of
+    select_plan and sparse_attention.  o_host is readable once `stream` has completed.
+    """
+    import torch
+
+    _check_bf16(q, k, v, o)
+    for t in (q_host, k_host, v_host, o_host):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("host tensors must be contiguous bf16 CPU tensors shaped like q")
+    cin = None if copy_in_stream is None else copy_in_stream.cuda_stream
+    cout = None if copy_out_stream is None else copy_out_stream.cuda_stream
+    _abi.check(absa_step_host(p, _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host), _ptr(q),
+                              _ptr(k), _ptr(v), _ptr(o), _ptr(scores), plan.c, _ptr(ws),
+                              ws.numel(), int(heads_per_run), _stream_handle(stream), cin, cout),
+               "absa_step_host")
+    return o_host

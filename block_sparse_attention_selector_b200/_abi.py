@@ -27,7 +27,7 @@ EXPORTED = (
     "absa_version", "absa_status_string", "absa_check_params", "absa_plan_capacity",
     "absa_workspace_bytes", "absa_select_scores", "absa_sample_plan", "absa_select_plan",
     "absa_sparse_attention", "absa_dense_reference", "absa_plan_check",
-    "absa_select_scores_static",
+    "absa_select_scores_static", "absa_step_host",
 )
 
 ABSA_STATIC_SCRATCH_BYTES = 64 << 20
@@ -97,6 +97,9 @@ def lib():
         L.absa_plan_check.restype = st
         L.absa_select_scores_static.argtypes = [P, vp, vp, vp, vp]
         L.absa_select_scores_static.restype = st
+        L.absa_step_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, Q, vp, sz,
+                                     ctypes.c_int32, vp, vp, vp]
+        L.absa_step_host.restype = st
         _lib = L
     return _lib
 
@@ -155,3 +158,10 @@ def absa_plan_check(plan, stream):
 def absa_select_scores_static(p, q, k, scores, stream):
     """Selector scores with the library's built-in scratch (no workspace argument)."""
     return lib().absa_select_scores_static(ctypes.byref(p), q, k, scores, stream)
+
+
+def absa_step_host(p, q_host, k_host, v_host, o_host, q, k, v, o, scores, plan, ws, ws_bytes,
+                   heads_per_run, stream, copy_in_stream, copy_out_stream):
+    return lib().absa_step_host(ctypes.byref(p), q_host, k_host, v_host, o_host, q, k, v, o,
+                                scores, ctypes.byref(plan), ws, ws_bytes, heads_per_run, stream,
+                                copy_in_stream, copy_out_stream)

@@ -2,7 +2,10 @@
 // workspace layout, tensor maps for the TMA loads, and kernel launches on the
 // caller's stream.  No allocation, no synchronisation (except absa_plan_check).
 #include <math.h>
+
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "absa_kernels.cuh"
 
@@ -162,6 +165,89 @@ size_t absa_workspace_bytes(const absa_params *p) {
 
 namespace {
 
+// A run of whole heads: flattened (b, h) rows bh0 .. bh0 + nbh - 1.  Every
+// stage works per head (pooling, k-means and the score softmax per head; plan
+// rows and attention per (head, query block)), so a run computes exactly the
+// values of those heads in a call over all of them.
+struct HeadRun {
+    int64_t bh0, nbh;
+};
+
+HeadRun all_heads(const absa_params *p) { return HeadRun{0, (int64_t)p->B * p->H}; }
+
+// Stages without argument checks (the callers check once).
+absa_status select_scores_run(const absa_params *p, const void *q, const void *k, float *scores,
+                              void *ws, int32_t *status, HeadRun hr, cudaStream_t s) {
+    const WsLayout L = ws_layout(p);
+    const Dims dm = dims_of(p);
+    const int64_t d = p->d;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    auto *kb_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_hi) + hr.bh0 * dm.nkb * d;
+    auto *kb_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_lo) + hr.bh0 * dm.nkb * d;
+    auto *mu = reinterpret_cast<float *>(w8 + L.mu) + hr.bh0 * dm.nqb * 8 * d;
+    auto *mu_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_hi) + hr.bh0 * dm.nqb * 8 * d;
+    auto *mu_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_lo) + hr.bh0 * dm.nqb * 8 * d;
+    auto *w = reinterpret_cast<float *>(w8 + L.w) + hr.bh0 * dm.nqb * 8;
+    auto *assign = w8 + L.assign + hr.bh0 * dm.nqb * 128;
+    const auto *qh = static_cast<const __nv_bfloat16 *>(q) + hr.bh0 * p->N * d;
+    const auto *kh = static_cast<const __nv_bfloat16 *>(k) + hr.bh0 * p->N * d;
+    float *sh = scores + hr.bh0 * dm.nqb * (int64_t)dm.nkb;
+
+    CUtensorMap tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo;
+    if (!make_map_bf16(&tm_kb_hi, kb_hi, hr.nbh * dm.nkb, p->d) ||
+        !make_map_bf16(&tm_kb_lo, kb_lo, hr.nbh * dm.nkb, p->d) ||
+        !make_map_bf16(&tm_mu_hi, mu_hi, hr.nbh * dm.nqb * 8, p->d) ||
+        !make_map_bf16(&tm_mu_lo, mu_lo, hr.nbh * dm.nqb * 8, p->d))
+        return ABSA_ERR_CUDA;
+
+    cudaError_t e = launch_pool(kh, kb_hi, kb_lo, hr.nbh, p->N, dm.nkb, p->d, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = launch_kmeans(qh, hr.nbh, p->N, dm.nqb, p->d, p->kmeans_iters, mu, mu_hi, mu_lo, w, assign,
+                      s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, sh, hr.nbh, dm.nqb, dm.nkb, p->d,
+                     p->softmax_scale, status, s);
+    return from_cuda(e);
+}
+
+absa_status sample_plan_run(const absa_params *p, const float *scores, const absa_plan *plan,
+                            HeadRun hr, cudaStream_t s) {
+    const Dims dm = dims_of(p);
+    const int64_t row0 = hr.bh0 * dm.nqb, cap = plan->capacity;
+    return from_cuda(launch_sample(scores + row0 * dm.nkb, hr.nbh * dm.nqb, dm.nkb,
+                                   p->budget_blocks, p->seed, plan->capacity, plan->counts + row0,
+                                   plan->kv_index + row0 * cap, plan->log_pi + row0 * cap,
+                                   plan->r_R + 2 * row0, plan->status, row0, s));
+}
+
+absa_status attention_run(const absa_params *p, const void *q, const void *k, const void *v,
+                          const absa_plan *plan, void *o, int32_t *status, HeadRun hr,
+                          cudaStream_t s) {
+    const Dims dm = dims_of(p);
+    const int64_t off = hr.bh0 * p->N * (int64_t)p->d;
+    const auto *qh = static_cast<const __nv_bfloat16 *>(q) + off;
+    const auto *kh = static_cast<const __nv_bfloat16 *>(k) + off;
+    const auto *vh = static_cast<const __nv_bfloat16 *>(v) + off;
+    auto *oh = static_cast<__nv_bfloat16 *>(o) + off;
+    const bool dense = plan == nullptr;
+    CUtensorMap tq, tk, tv;
+    // sparse gathers: one 4-row box (one 4-token block) per 64-column region
+    const int kv_box = dense ? 128 : 4;
+    if (!make_map_bf16(&tq, qh, hr.nbh * p->N, p->d) ||
+        !make_map_bf16(&tk, kh, hr.nbh * p->N, p->d, kv_box) ||
+        !make_map_bf16(&tv, vh, hr.nbh * p->N, p->d, kv_box))
+        return ABSA_ERR_CUDA;
+    if (dense)
+        return from_cuda(launch_attention(true, tq, tk, tv, kh, vh, oh, hr.nbh, p->N, dm.nqb,
+                                          dm.nkb, p->d, p->softmax_scale, nullptr, nullptr,
+                                          nullptr, 0, status, s));
+    const int64_t row0 = hr.bh0 * dm.nqb, cap = plan->capacity;
+    return from_cuda(launch_attention(false, tq, tk, tv, kh, vh, oh, hr.nbh, p->N, dm.nqb,
+                                      dm.nkb, p->d, p->softmax_scale, plan->counts + row0,
+                                      plan->kv_index + row0 * cap, plan->log_pi + row0 * cap,
+                                      plan->capacity, plan->status, s));
+}
+
 absa_status select_scores_impl(const absa_params *p, const void *q, const void *k, float *scores,
                                void *ws, size_t ws_bytes, int32_t *status, void *stream) {
     absa_status st = absa_check_params(p);
@@ -169,35 +255,9 @@ absa_status select_scores_impl(const absa_params *p, const void *q, const void *
     if (!q || !k || !scores || !ws) return ABSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || !aligned16(ws))
         return ABSA_ERR_INVALID_ARG;
-    const WsLayout L = ws_layout(p);
-    if (ws_bytes < L.total) return ABSA_ERR_WORKSPACE;
-    const Dims dm = dims_of(p);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    uint8_t *w8 = static_cast<uint8_t *>(ws);
-    auto *kb_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_hi);
-    auto *kb_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_lo);
-    auto *mu = reinterpret_cast<float *>(w8 + L.mu);
-    auto *mu_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_hi);
-    auto *mu_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_lo);
-    auto *w = reinterpret_cast<float *>(w8 + L.w);
-    auto *assign = w8 + L.assign;
-
-    CUtensorMap tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo;
-    if (!make_map_bf16(&tm_kb_hi, kb_hi, dm.BH * dm.nkb, p->d) ||
-        !make_map_bf16(&tm_kb_lo, kb_lo, dm.BH * dm.nkb, p->d) ||
-        !make_map_bf16(&tm_mu_hi, mu_hi, dm.BH * dm.nqb * 8, p->d) ||
-        !make_map_bf16(&tm_mu_lo, mu_lo, dm.BH * dm.nqb * 8, p->d))
-        return ABSA_ERR_CUDA;
-
-    cudaError_t e = launch_pool(static_cast<const __nv_bfloat16 *>(k), kb_hi, kb_lo, dm.BH, p->N,
-                                dm.nkb, p->d, s);
-    if (e != cudaSuccess) return from_cuda(e);
-    e = launch_kmeans(static_cast<const __nv_bfloat16 *>(q), dm.BH, p->N, dm.nqb, p->d,
-                      p->kmeans_iters, mu, mu_hi, mu_lo, w, assign, s);
-    if (e != cudaSuccess) return from_cuda(e);
-    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, scores, dm.BH, dm.nqb, dm.nkb,
-                     p->d, p->softmax_scale, status, s);
-    return from_cuda(e);
+    if (ws_bytes < ws_layout(p).total) return ABSA_ERR_WORKSPACE;
+    return select_scores_run(p, q, k, scores, ws, status, all_heads(p),
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 absa_status sample_plan_impl(const absa_params *p, const float *scores, const absa_plan *plan,
@@ -207,16 +267,12 @@ absa_status sample_plan_impl(const absa_params *p, const float *scores, const ab
     if (!scores || !aligned16(scores)) return ABSA_ERR_INVALID_ARG;
     st = check_plan(p, plan);
     if (st != ABSA_OK) return st;
-    const Dims dm = dims_of(p);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaSuccess;
     if (reset_status) {
-        e = cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s);
+        cudaError_t e = cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s);
         if (e != cudaSuccess) return from_cuda(e);
     }
-    e = launch_sample(scores, dm.BH * dm.nqb, dm.nkb, p->budget_blocks, p->seed, plan->capacity,
-                      plan->counts, plan->kv_index, plan->log_pi, plan->r_R, plan->status, s);
-    return from_cuda(e);
+    return sample_plan_run(p, scores, plan, all_heads(p), s);
 }
 
 // Built-in workspace of absa_select_scores_static: one copy per device for as
@@ -289,18 +345,8 @@ absa_status absa_sparse_attention(const absa_params *p, const void *q, const voi
     if (!q || !k || !v || !o) return ABSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
         return ABSA_ERR_INVALID_ARG;
-    const Dims dm = dims_of(p);
-    CUtensorMap tq, tk, tv;
-    // sparse gathers: one 4-row box (one 4-token block) per 64-column region
-    if (!make_map_bf16(&tq, q, dm.BH * p->N, p->d) || !make_map_bf16(&tk, k, dm.BH * p->N, p->d, 4) ||
-        !make_map_bf16(&tv, v, dm.BH * p->N, p->d, 4))
-        return ABSA_ERR_CUDA;
-    return from_cuda(launch_attention(false, tq, tk, tv, static_cast<const __nv_bfloat16 *>(k),
-                                      static_cast<const __nv_bfloat16 *>(v),
-                                      static_cast<__nv_bfloat16 *>(o), dm.BH,
-                                      p->N, dm.nqb, dm.nkb, p->d, p->softmax_scale, plan->counts,
-                                      plan->kv_index, plan->log_pi, plan->capacity, plan->status,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+    return attention_run(p, q, k, v, plan, o, plan->status, all_heads(p),
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,
@@ -311,17 +357,81 @@ absa_status absa_dense_reference(const absa_params *p, const void *q, const void
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
         return ABSA_ERR_INVALID_ARG;
     if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return ABSA_ERR_INVALID_ARG;
-    const Dims dm = dims_of(p);
-    CUtensorMap tq, tk, tv;
-    if (!make_map_bf16(&tq, q, dm.BH * p->N, p->d) || !make_map_bf16(&tk, k, dm.BH * p->N, p->d) ||
-        !make_map_bf16(&tv, v, dm.BH * p->N, p->d))
-        return ABSA_ERR_CUDA;
-    return from_cuda(launch_attention(true, tq, tk, tv, static_cast<const __nv_bfloat16 *>(k),
-                                      static_cast<const __nv_bfloat16 *>(v),
-                                      static_cast<__nv_bfloat16 *>(o), dm.BH,
-                                      p->N, dm.nqb, dm.nkb, p->d, p->softmax_scale, nullptr,
-                                      nullptr, nullptr, 0, status,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+    return attention_run(p, q, k, v, nullptr, o, status, all_heads(p),
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+absa_status absa_step_host(const absa_params *p, const void *q_host, const void *k_host,
+                           const void *v_host, void *o_host, void *q, void *k, void *v, void *o,
+                           float *scores, const absa_plan *plan, void *ws, size_t ws_bytes,
+                           int32_t heads_per_run, void *stream, void *copy_in_stream,
+                           void *copy_out_stream) {
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    st = check_plan(p, plan);
+    if (st != ABSA_OK) return st;
+    if (!q_host || !k_host || !v_host || !o_host || !q || !k || !v || !o || !scores || !ws)
+        return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(scores) ||
+        !aligned16(ws))
+        return ABSA_ERR_INVALID_ARG;
+    if (heads_per_run < 1) return ABSA_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(p).total) return ABSA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t s_in = copy_in_stream ? reinterpret_cast<cudaStream_t>(copy_in_stream) : s;
+    cudaStream_t s_out = copy_out_stream ? reinterpret_cast<cudaStream_t>(copy_out_stream) : s;
+    const int64_t BH = (int64_t)p->B * p->H;
+    const size_t head_bytes = (size_t)p->N * (size_t)p->d * 2;
+
+    std::vector<cudaEvent_t> events;
+    auto event = [&](cudaEvent_t *ev) {
+        if (cudaEventCreateWithFlags(ev, cudaEventDisableTiming) != cudaSuccess) return false;
+        events.push_back(*ev);
+        return true;
+    };
+    // Recorded events may be destroyed before they complete: their resources
+    // are released once the device reaches them.
+    auto finish = [&](absa_status r) {
+        for (cudaEvent_t ev : events) cudaEventDestroy(ev);
+        return r;
+    };
+
+    // copies into q/k/v start only after earlier work on `stream` (which may
+    // still read those buffers) has finished
+    cudaEvent_t ev;
+    if (!event(&ev) || cudaEventRecord(ev, s) != cudaSuccess ||
+        cudaStreamWaitEvent(s_in, ev, 0) != cudaSuccess ||
+        cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s) != cudaSuccess)
+        return finish(ABSA_ERR_CUDA);
+    for (int64_t bh0 = 0; bh0 < BH; bh0 += heads_per_run) {
+        const HeadRun hr{bh0, std::min<int64_t>(heads_per_run, BH - bh0)};
+        const size_t off = (size_t)bh0 * head_bytes, bytes = (size_t)hr.nbh * head_bytes;
+        const void *src[3] = {q_host, k_host, v_host};
+        void *dst[3] = {q, k, v};
+        for (int i = 0; i < 3; ++i)
+            if (cudaMemcpyAsync(static_cast<uint8_t *>(dst[i]) + off,
+                                static_cast<const uint8_t *>(src[i]) + off, bytes,
+                                cudaMemcpyHostToDevice, s_in) != cudaSuccess)
+                return finish(ABSA_ERR_CUDA);
+        if (!event(&ev) || cudaEventRecord(ev, s_in) != cudaSuccess ||
+            cudaStreamWaitEvent(s, ev, 0) != cudaSuccess)
+            return finish(ABSA_ERR_CUDA);
+        st = select_scores_run(p, q, k, scores, ws, plan->status, hr, s);
+        if (st == ABSA_OK) st = sample_plan_run(p, scores, plan, hr, s);
+        if (st == ABSA_OK) st = attention_run(p, q, k, v, plan, o, plan->status, hr, s);
+        if (st != ABSA_OK) return finish(st);
+        if (!event(&ev) || cudaEventRecord(ev, s) != cudaSuccess ||
+            cudaStreamWaitEvent(s_out, ev, 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<uint8_t *>(o_host) + off,
+                            static_cast<const uint8_t *>(o) + off, bytes, cudaMemcpyDeviceToHost,
+                            s_out) != cudaSuccess)
+            return finish(ABSA_ERR_CUDA);
+    }
+    // `stream` completes after the last output copy
+    if (!event(&ev) || cudaEventRecord(ev, s_out) != cudaSuccess ||
+        cudaStreamWaitEvent(s, ev, 0) != cudaSuccess)
+        return finish(ABSA_ERR_CUDA);
+    return finish(ABSA_OK);
 }
 
 absa_status absa_plan_check(const absa_plan *plan, void *stream) {

@@ -71,7 +71,9 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
     }
 }
 
-// One CTA per plan row (b,h,qb).  Key blocks are handled in groups of 32 (one
+// One CTA per plan row (b,h,qb); the grid covers rows row0 .. row0+gridDim-1
+// of the whole problem (scores and plan pointers start at row0, the hash
+// counter uses the global row).  Key blocks are handled in groups of 32 (one
 // per lane); warp w owns a contiguous run of groups, so the taken blocks of
 // warp w all precede those of warp w+1 and one scan of the 8 warp counts
 // places every entry.  Shared memory: q_j - 1 as u32 per block, one capped
@@ -87,7 +89,7 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
 __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
-    uint64_t *__restrict__ r_R, int32_t *status) {
+    uint64_t *__restrict__ r_R, int32_t *status, int64_t row0) {
     extern __shared__ __align__(16) uint32_t samp_smem[];
     const int ngroups = (nkb + 31) >> 5;
     uint32_t *qm1 = samp_smem;                      // [ngroups*32]
@@ -260,8 +262,9 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
 
     // Poisson draws: one taken word per group; SplitMix64 state of block j is
-    // base + j * gamma with base = mix(seed) + (row * NKB + 1) * gamma
-    const uint64_t base = splitmix64_mix(seed) + ((uint64_t)row * (uint64_t)nkb + 1) * kGamma;
+    // base + j * gamma with base = mix(seed) + (global row * NKB + 1) * gamma
+    const uint64_t base =
+        splitmix64_mix(seed) + ((uint64_t)(row0 + row) * (uint64_t)nkb + 1) * kGamma;
     const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
     int taken = 0;
     uint64_t state = base + (uint64_t)(g0 * 32 + lane) * kGamma;  // state of block j
@@ -325,14 +328,14 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
 
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
                           int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
-                          uint64_t *r_R, int32_t *status, cudaStream_t stream) {
+                          uint64_t *r_R, int32_t *status, int64_t row0, cudaStream_t stream) {
     const int ngroups = (nkb + 31) / 32;
     const int smem = (ngroups * 32 + 2 * ngroups + kCandMax) * 4;
     cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     absa_sample_kernel<<<(unsigned)rows, kSampleThreads, smem, stream>>>(
-        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status);
+        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0);
     return cudaGetLastError();
 }
 

@@ -187,6 +187,37 @@ absa_status absa_dense_reference(const absa_params *p, const void *q, const void
 absa_status absa_select_scores_static(const absa_params *p, const void *q, const void *k,
                                       float *scores, void *stream);
 
+/* One whole step on host tensors, pipelined over runs of heads (no
+ * counterpart on the pages: a library-interface addition for callers whose
+ * q, k, v live in host memory).  For each run of heads_per_run flattened
+ * (b,h) heads: copy its q, k, v rows from q_host/k_host/v_host (bf16
+ * [B,H,N,d], same layout as on the device) into q/k/v on copy_in_stream,
+ * then on `stream` run the selector, the sampler and the sparse attention for
+ * those heads, then copy its o rows back into o_host on copy_out_stream.  The
+ * copies of one run overlap the compute of the others.  Heads are
+ * independent in every stage and the draw counter uses the global plan row,
+ * so scores, plan and o equal those of absa_select_plan followed by
+ * absa_sparse_attention on the whole problem, for any heads_per_run >= 1.
+ *  - q, k, v, o, scores, plan, ws: device buffers as in those calls (caller
+ *    owned; q/k/v are overwritten with the host inputs).  ws must hold
+ *    absa_workspace_bytes(p) bytes.
+ *  - Host buffers must stay valid until the step completes; page-locked host
+ *    memory (cudaHostAlloc / cudaHostRegister) is needed for the copies to
+ *    overlap, pageable memory gives the same results without overlap.
+ *  - copy_in_stream / copy_out_stream may be NULL (then `stream` does the
+ *    copies, with no overlap).  Copies into q/k/v wait for the work enqueued
+ *    on `stream` before the call; `stream` completes after the last output
+ *    copy, so synchronising `stream` makes o_host readable.
+ *  - Resets plan->status first.  Creates two CUDA events per run and
+ *    destroys them before returning (no device memory is allocated).
+ *  - Host-detectable errors return before anything is enqueued; a failing
+ *    CUDA call returns ABSA_ERR_CUDA with the earlier runs enqueued. */
+absa_status absa_step_host(const absa_params *p, const void *q_host, const void *k_host,
+                           const void *v_host, void *o_host, void *q, void *k, void *v, void *o,
+                           float *scores, const absa_plan *plan, void *ws, size_t ws_bytes,
+                           int32_t heads_per_run, void *stream, void *copy_in_stream,
+                           void *copy_out_stream);
+
 /* Synchronise `stream`, read plan->status and map it to a status code
  * (TIMEOUT > BAD_PLAN > OVERFLOW > OK).  Does not clear the word. */
 absa_status absa_plan_check(const absa_plan *plan, void *stream);

@@ -102,6 +102,19 @@ def test_entry_points_reject_null_and_misaligned_pointers_before_cuda(L):
     bad = _abi.absa_plan(5, 128, 96, 16, 16, 16, 16, 16)
     assert _abi.absa_sparse_attention(p, 16, 16, 16, bad, 16, None) == _abi.ABSA_ERR_INVALID_ARG
     assert _abi.absa_plan_check(_abi.absa_plan(), None) == _abi.ABSA_ERR_INVALID_ARG
+    # the host-buffer step: null host pointers, an empty head run, a short workspace
+    good = _abi.absa_plan(4, 128, 96, 16, 16, 16, 16, 16)
+    step = _abi.absa_step_host
+    assert step(p, None, 16, 16, 16, 16, 16, 16, 16, 16, good, 16, ws, 4, None, None,
+                None) == _abi.ABSA_ERR_INVALID_ARG
+    assert step(p, 16, 16, 16, 16, 16, 16, 8, 16, 16, good, 16, ws, 4, None, None,
+                None) == _abi.ABSA_ERR_INVALID_ARG
+    assert step(p, 16, 16, 16, 16, 16, 16, 16, 16, 16, good, 16, ws, 0, None, None,
+                None) == _abi.ABSA_ERR_INVALID_ARG
+    assert step(p, 16, 16, 16, 16, 16, 16, 16, 16, 16, good, 16, ws - 1, 4, None, None,
+                None) == _abi.ABSA_ERR_WORKSPACE
+    assert step(p, 16, 16, 16, 16, 16, 16, 16, 16, 16, bad, 16, ws, 4, None, None,
+                None) == _abi.ABSA_ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
