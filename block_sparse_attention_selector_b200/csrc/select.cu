@@ -62,29 +62,40 @@ __global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__r
 // ------------------------------------------------------------------------ K2
 
 // One CTA (128 threads) per query block.  fp32 arithmetic in a fixed order:
+//  load:                  every thread issues all of its 16-byte loads of the
+//                         block before storing any of them (one memory
+//                         latency per block), into rows of pitch D+8 bf16
+//                         (an odd number of 16-byte units, so 8 threads
+//                         reading 16 bytes of 8 different rows hit 8
+//                         different bank groups);
 //  assignment (thread i): dist_c = sum over ascending e of fma(x-mu, x-mu, .),
 //                         two clusters per packed f32x2 instruction (each lane
 //                         rounds exactly like the scalar operation), argmin
-//                         with ties to the lowest c;
-//  update     (thread e): members of each cluster ranked in ascending i with
-//                         warp ballots, member sums over ascending i read from
-//                         the bf16 copy of the block in shared memory (no bank
-//                         conflicts: a warp reads 32 consecutive columns of one
-//                         row), mu = sum / count (IEEE division); an empty
-//                         cluster keeps mu.
+//                         with ties to the lowest c; row i is read 8 dims at
+//                         a time;
+//  update:                members of each cluster ranked in ascending i with
+//                         warp ballots; the clusters are split in contiguous
+//                         runs of about equal membership over 256/D groups of
+//                         D/2 threads, thread dl of a group summing dims 2dl
+//                         and 2dl+1 (one bf16 pair of each member row) over
+//                         ascending i, with the next 8 members' loads in
+//                         flight while the current 8 are added;
+//                         mu = sum / count (IEEE division); an empty cluster
+//                         keeps mu.
 template <int D>
 struct KmeansSmem {
-    static constexpr int kRow = D + 2;                  // bf16 row pitch: 4*(D/2+1) bytes, so
-                                                        // thread i reading row i is conflict-free
-    static constexpr int kX = 0;                        // bf16 [128][D+2]
+    static constexpr int kRow = D + 8;                  // bf16 row pitch: an odd number of 16 B units
+    static constexpr int kX = 0;                        // bf16 [128][D+8]
     static constexpr int kMu = kX + 128 * kRow * 2;     // f32 [D][8] (transposed)
     static constexpr int kList = kMu + D * 8 * 4;       // i32 [8][128] member lists
     static constexpr int kCnt = kList + 8 * 128 * 4;    // i32 [4 warps][8] + [8] totals
     static constexpr int kBytes = kCnt + (4 * 8 + 8) * 4;
+    static_assert(((kRow * 2 / 16) & 1) == 1 && (kRow * 2) % 16 == 0, "row pitch");
+    static_assert(kMu % 16 == 0 && kList % 16 == 0, "alignment");
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) absa_kmeans_kernel(
+__global__ void __launch_bounds__(128, 4) absa_kmeans_kernel(
     const __nv_bfloat16 *__restrict__ q, int N, int nqb, int iters, float *__restrict__ mu_out,
     __nv_bfloat16 *__restrict__ mu_hi, __nv_bfloat16 *__restrict__ mu_lo, float *__restrict__ w_out,
     uint8_t *__restrict__ assign_out) {
@@ -104,13 +115,21 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     const int m = min(128, N - qb * 128);
     const __nv_bfloat16 *src = q + (bh * N + (int64_t)qb * 128) * D;
 
-    constexpr int XR = S::kRow;
+    constexpr int XR = S::kRow;      // bf16 per row
+    constexpr int XW = XR / 2;       // 32-bit words per row
+    constexpr int CPR = D / 8;       // 16-byte units per row of q
     {
-        const uint32_t *src32 = reinterpret_cast<const uint32_t *>(src);
-        uint32_t *xs32 = reinterpret_cast<uint32_t *>(xs);
-        for (int idx = tid; idx < m * (D / 2); idx += 128) {
-            const int r = idx / (D / 2), w = idx % (D / 2);
-            xs32[r * (XR / 2) + w] = __ldg(src32 + idx);
+        const uint4 *src4 = reinterpret_cast<const uint4 *>(src);
+        uint4 v[CPR];
+#pragma unroll
+        for (int u = 0; u < CPR; ++u) {  // 128 * CPR units, CPR per thread
+            const int idx = tid + 128 * u;
+            if (idx / CPR < m) v[u] = __ldg(src4 + idx);
+        }
+#pragma unroll
+        for (int u = 0; u < CPR; ++u) {
+            const int idx = tid + 128 * u, r = idx / CPR, c = idx % CPR;
+            if (r < m) *reinterpret_cast<uint4 *>(xs + r * XR + c * 8) = v[u];
         }
     }
     __syncthreads();
@@ -120,18 +139,21 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
     }
     __syncthreads();
 
+    const uint32_t *xs32 = reinterpret_cast<const uint32_t *>(xs);
     for (int it = 0; it < iters; ++it) {
         int a = 0;
         if (tid < m) {
             uint64_t dist[NC / 2] = {0, 0, 0, 0};  // (+0.f, +0.f) pairs
-            const uint32_t *xrow = reinterpret_cast<const uint32_t *>(xs + tid * XR);
-#pragma unroll 4
-            for (int e2 = 0; e2 < D / 2; ++e2) {
-                const uint32_t pair = xrow[e2];
+            const __nv_bfloat16 *xrow = xs + tid * XR;
+#pragma unroll 2
+            for (int c8 = 0; c8 < CPR; ++c8) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xrow + c8 * 8);
+                const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int e = 2 * e2 + h;
-                    const uint32_t xb = h ? (pair & 0xFFFF0000u) : (pair << 16);
+                for (int h = 0; h < 8; ++h) {
+                    const int e = c8 * 8 + h;
+                    const uint32_t pair = wv[h >> 1];
+                    const uint32_t xb = (h & 1) ? (pair & 0xFFFF0000u) : (pair << 16);
                     const uint64_t x2 = (uint64_t)xb | ((uint64_t)xb << 32);
                     const ulonglong2 m01 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC);
                     const ulonglong2 m45 = *reinterpret_cast<const ulonglong2 *>(mut + e * NC + 4);
@@ -170,23 +192,53 @@ __global__ void __launch_bounds__(128) absa_kmeans_kernel(
         }
         if (tid < NC) cnt_s[tid] = wcnt[tid] + wcnt[NC + tid] + wcnt[2 * NC + tid] + wcnt[3 * NC + tid];
         __syncthreads();
-        if (tid < D) {
+        {
+            constexpr int G = 256 / D;  // groups of D/2 threads (whole warps)
+            const int g = tid / (D / 2), dl = tid % (D / 2);
+            const uint32_t *xw = xs32 + dl;  // word dl of row 0
+            int before = 0;
 #pragma unroll 1
             for (int c = 0; c < NC; ++c) {
                 const int n = cnt_s[c];
-                if (n == 0) continue;
+                const int owner = min(G - 1, ((2 * before + n) * G) / (2 * m));
+                before += n;
+                if (n == 0 || owner != g) continue;
                 const int *ml = mlist + c * 128;
-                float acc = 0.f;
+                float acc0 = 0.f, acc1 = 0.f;
+                auto add8 = [&](const uint32_t (&pv)[8]) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        acc0 = __fadd_rn(acc0, __uint_as_float(pv[u] << 16));
+                        acc1 = __fadd_rn(acc1, __uint_as_float(pv[u] & 0xFFFF0000u));
+                    }
+                };
+                auto load8 = [&](int t0, uint32_t (&pv)[8]) {
+                    const int4 ia = *reinterpret_cast<const int4 *>(ml + t0);
+                    const int4 ib = *reinterpret_cast<const int4 *>(ml + t0 + 4);
+                    const int id[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) pv[u] = xw[id[u] * XW];
+                };
                 int t = 0;
-                for (; t + 4 <= n; t += 4) {  // loads ahead, adds in order
-                    const float x0 = __bfloat162float(xs[ml[t] * XR + tid]);
-                    const float x1 = __bfloat162float(xs[ml[t + 1] * XR + tid]);
-                    const float x2 = __bfloat162float(xs[ml[t + 2] * XR + tid]);
-                    const float x3 = __bfloat162float(xs[ml[t + 3] * XR + tid]);
-                    acc = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(acc, x0), x1), x2), x3);
+                if (n >= 8) {
+                    uint32_t cur[8];
+                    load8(0, cur);
+                    for (t = 8; t + 8 <= n; t += 8) {
+                        uint32_t nxt[8];
+                        load8(t, nxt);
+                        add8(cur);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
+                    }
+                    add8(cur);
                 }
-                for (; t < n; ++t) acc = __fadd_rn(acc, __bfloat162float(xs[ml[t] * XR + tid]));
-                mut[tid * NC + c] = __fdiv_rn(acc, (float)n);
+                for (; t < n; ++t) {
+                    const uint32_t pv = xw[ml[t] * XW];
+                    acc0 = __fadd_rn(acc0, __uint_as_float(pv << 16));
+                    acc1 = __fadd_rn(acc1, __uint_as_float(pv & 0xFFFF0000u));
+                }
+                mut[(2 * dl) * NC + c] = __fdiv_rn(acc0, (float)n);
+                mut[(2 * dl + 1) * NC + c] = __fdiv_rn(acc1, (float)n);
             }
         }
         __syncthreads();
