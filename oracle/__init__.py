@@ -55,6 +55,13 @@ def lib():
         L.oracle_sample_plan.argtypes = [_i32, _i32, _i32, _i32, _i64, _u64, _f32p, _i32, _i32p,
                                          _i32p, _f32p, _u64p]
         L.oracle_sample_plan.restype = _i32
+        L.oracle_sample_plan_design.argtypes = L.oracle_sample_plan.argtypes + [_i32]
+        L.oracle_sample_plan_design.restype = _i32
+        L.oracle_systematic_take.argtypes = [_f32p, _i32, _i64, ctypes.c_uint32, _u8p,
+                                             ctypes.POINTER(_u64), ctypes.POINTER(_u64)]
+        L.oracle_systematic_take.restype = _i32
+        L.oracle_sample_row_systematic.argtypes = L.oracle_sample_row.argtypes
+        L.oracle_sample_row_systematic.restype = _i32
         L.oracle_sparse_attention.argtypes = [_i32, _i32, _i64, _i32, _dbl, _u16p, _u16p, _u16p,
                                               _i32, _i32, _i32p, _i32p, _f32p, _i32, _i32, _f64p]
         L.oracle_num_threads.restype = _i32
@@ -135,15 +142,19 @@ def draw_u32(seed, ctr):
     return int(lib().oracle_draw_u32(seed & 0xFFFFFFFFFFFFFFFF, ctr & 0xFFFFFFFFFFFFFFFF))
 
 
-def sample_row(s, n, seed, row, cap):
-    """SIP plan of one score row -> (kv_index, log_pi, taken, r, R)."""
+def sample_row(s, n, seed, row, cap, design="poisson"):
+    """SIP plan of one score row -> (kv_index, log_pi, taken, r, R).
+
+    design: "poisson" (independent draws) or "systematic" (exactly n blocks)."""
     s = _c(s, np.float32)
     idx = np.zeros(cap, np.int32)
     lp = np.zeros(cap, np.float32)
     r = _u64()
     R = _u64()
-    taken = lib().oracle_sample_row(s, s.shape[0], int(n), int(seed), int(row), int(cap), idx, lp,
-                                    ctypes.byref(r), ctypes.byref(R))
+    fn = {"poisson": lib().oracle_sample_row,
+          "systematic": lib().oracle_sample_row_systematic}[design]
+    taken = fn(s, s.shape[0], int(n), int(seed), int(row), int(cap), idx, lp, ctypes.byref(r),
+               ctypes.byref(R))
     m = min(taken, cap)
     return idx[:m].copy(), lp[:m].copy(), int(taken), int(r.value), int(R.value)
 
@@ -209,10 +220,23 @@ def select_scores(q, k, nc=8, iters=3, scale=None, qb_range=(0, 0)):
     return scores, mu, w, assign
 
 
-def sample_plan(scores, n, seed, cap):
+def systematic_take(s, n, U):
+    """Systematic design on one score row with the uniform U (u32) given:
+    -> (take bool[nkb], r, R)."""
+    s = _c(s, np.float32)
+    take = np.zeros(s.shape[0], np.uint8)
+    r = _u64()
+    R = _u64()
+    lib().oracle_systematic_take(s, s.shape[0], int(n), int(U) & 0xFFFFFFFF, take,
+                                 ctypes.byref(r), ctypes.byref(R))
+    return take.astype(bool), int(r.value), int(R.value)
+
+
+def sample_plan(scores, n, seed, cap, design="poisson"):
     """SIP plan for every row of a [B,H,NQB,NKB] fp32 score array.
 
-    Returns dict(counts, kv_index, log_pi, r_R, overflow_rows).
+    design: "poisson" or "systematic".  Returns dict(counts, kv_index, log_pi, r_R,
+    overflow_rows).
     """
     scores = _c(scores, np.float32)
     B, H, nqb, nkb = scores.shape
@@ -220,8 +244,9 @@ def sample_plan(scores, n, seed, cap):
     idx = np.zeros((B, H, nqb, cap), np.int32)
     lp = np.zeros((B, H, nqb, cap), np.float32)
     r_R = np.zeros((B, H, nqb, 2), np.uint64)
-    ov = lib().oracle_sample_plan(B, H, nqb, nkb, int(n), int(seed), scores, int(cap), counts, idx,
-                                  lp, r_R)
+    ov = lib().oracle_sample_plan_design(B, H, nqb, nkb, int(n), int(seed), scores, int(cap),
+                                         counts, idx, lp, r_R,
+                                         {"poisson": 0, "systematic": 1}[design])
     return dict(counts=counts, kv_index=idx, log_pi=lp, r_R=r_R, overflow_rows=int(ov))
 
 

@@ -248,6 +248,68 @@ int oracle_sample_row(const float *s, int nkb, int64_t n, uint64_t seed,
     return taken;
 }
 
+/* Systematic (fixed-size) design, written from its definition: with the
+ * integer pi of oracle_pi_solve scaled by R (a_j = R if capped, r*q_j
+ * otherwise; sum a_j = n*R), lay the blocks end to end on [0, n*R) in
+ * ascending j and put n points at (k + U/2^32)*R, k = 0..n-1.  Block j is
+ * taken iff a point falls in its interval [A_j, A_j + a_j), A_j = sum_{i<j} a_i.
+ * Each interval is at most R long, so it holds at most one point, block j is
+ * taken with probability a_j/R = pi_j over U, and exactly n blocks are taken.
+ * Arithmetic in units of R/2^32: point k sits at k*R*2^32 + U*R. */
+int oracle_systematic_take(const float *s, int nkb, int64_t n, uint32_t U,
+                           uint8_t *take, uint64_t *r_out, uint64_t *R_out)
+{
+    uint8_t *capped = (uint8_t *)malloc((size_t)nkb);
+    uint64_t r, R;
+    oracle_pi_solve(s, nkb, n, capped, &r, &R);
+    const unsigned __int128 period = (unsigned __int128)R << 32;
+    const unsigned __int128 phase = (unsigned __int128)U * R;
+    unsigned __int128 A = 0;  /* A_j * 2^32 */
+    int taken = 0;
+    for (int j = 0; j < nkb; ++j) {
+        const uint64_t a = capped[j] ? R : r * quantised_score(s[j]);
+        const unsigned __int128 lo = A, hi = A + ((unsigned __int128)a << 32);
+        /* first point at or after lo: k0 = ceil((lo - phase) / period) */
+        unsigned __int128 k0 = 0;
+        if (lo > phase)
+            k0 = (lo - phase + period - 1) / period;
+        take[j] = (k0 < (unsigned __int128)n) && (k0 * period + phase < hi);
+        taken += take[j];
+        A = hi;
+    }
+    free(capped);
+    *r_out = r;
+    *R_out = R;
+    return taken;
+}
+
+int oracle_sample_row_systematic(const float *s, int nkb, int64_t n, uint64_t seed,
+                                 uint64_t row, int cap, int32_t *kv_index, float *log_pi,
+                                 uint64_t *r_out, uint64_t *R_out)
+{
+    if (n >= nkb)
+        return oracle_sample_row(s, nkb, n, seed, row, cap, kv_index, log_pi, r_out, R_out);
+    uint8_t *take = (uint8_t *)malloc((size_t)nkb);
+    uint64_t r, R;
+    const uint32_t U = oracle_draw_u32(seed, row * (uint64_t)nkb);
+    oracle_systematic_take(s, nkb, n, U, take, &r, &R);
+    int taken = 0;
+    for (int j = 0; j < nkb; ++j) {
+        if (!take[j])
+            continue;
+        if (taken < cap) {
+            const uint64_t rq = r * quantised_score(s[j]);
+            kv_index[taken] = j;
+            log_pi[taken] = rq >= R ? 0.0f : (float)log((double)rq / (double)R);
+        }
+        taken += 1;
+    }
+    free(take);
+    *r_out = r;
+    *R_out = R;
+    return taken;
+}
+
 /* -------------------------------------------------------------- attention */
 
 static void attention_row(const float *qf, int d, const uint16_t *k,
@@ -406,18 +468,19 @@ void oracle_select_scores(int B, int H, int64_t N, int d, int nc, int iters,
     }
 }
 
-int oracle_sample_plan(int B, int H, int nqb, int nkb, int64_t n,
-                       uint64_t seed, const float *scores, int cap,
-                       int32_t *counts, int32_t *kv_index, float *log_pi,
-                       uint64_t *r_R)
+int oracle_sample_plan_design(int B, int H, int nqb, int nkb, int64_t n,
+                              uint64_t seed, const float *scores, int cap,
+                              int32_t *counts, int32_t *kv_index, float *log_pi,
+                              uint64_t *r_R, int systematic)
 {
     int overflow = 0;
     int64_t rows = (int64_t)B * H * nqb;
 #pragma omp parallel for schedule(dynamic, 16) reduction(+ : overflow)
     for (int64_t row = 0; row < rows; ++row) {
         uint64_t r, R;
-        int taken = oracle_sample_row(scores + row * nkb, nkb, n, seed, (uint64_t)row, cap,
-                                      kv_index + row * cap, log_pi + row * cap, &r, &R);
+        int taken = (systematic ? oracle_sample_row_systematic : oracle_sample_row)(
+            scores + row * nkb, nkb, n, seed, (uint64_t)row, cap, kv_index + row * cap,
+            log_pi + row * cap, &r, &R);
         counts[row] = taken < cap ? taken : cap;
         r_R[2 * row] = r;
         r_R[2 * row + 1] = R;
@@ -425,6 +488,14 @@ int oracle_sample_plan(int B, int H, int nqb, int nkb, int64_t n,
             overflow += 1;
     }
     return overflow;
+}
+
+int oracle_sample_plan(int B, int H, int nqb, int nkb, int64_t n, uint64_t seed,
+                       const float *scores, int cap, int32_t *counts, int32_t *kv_index,
+                       float *log_pi, uint64_t *r_R)
+{
+    return oracle_sample_plan_design(B, H, nqb, nkb, n, seed, scores, cap, counts, kv_index,
+                                     log_pi, r_R, 0);
 }
 
 void oracle_sparse_attention(int B, int H, int64_t N, int d, double scale,

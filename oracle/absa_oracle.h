@@ -93,6 +93,24 @@ int oracle_sample_row(const float *s, int nkb, int64_t n, uint64_t seed,
                       uint64_t row, int cap, int32_t *kv_index, float *log_pi,
                       uint64_t *r_out, uint64_t *R_out);
 
+/* Fixed-size alternative to the Poisson design (the SIP paragraph names no
+ * design): systematic sampling with probabilities pi.  Reading: the blocks
+ * are laid end to end in ascending j with lengths a_j = pi_j * R (a_j = R
+ * if capped, r*q_j otherwise), n points are placed at (k + U/2^32) * R for
+ * k = 0..n-1, and block j is taken iff a point falls in its interval.  Each
+ * block is taken with probability pi_j over U and exactly n blocks are
+ * taken.  take[nkb] (0/1); returns the number taken.  Requires
+ * 1 <= n < nkb. */
+int oracle_systematic_take(const float *s, int nkb, int64_t n, uint32_t U,
+                           uint8_t *take, uint64_t *r_out, uint64_t *R_out);
+
+/* Plan row of the systematic design: U = oracle_draw_u32(seed, row*nkb)
+ * (the counter of block 0 of the row), entries and log_pi as in
+ * oracle_sample_row; n >= nkb takes every block. */
+int oracle_sample_row_systematic(const float *s, int nkb, int64_t n, uint64_t seed,
+                                 uint64_t row, int cap, int32_t *kv_index, float *log_pi,
+                                 uint64_t *r_out, uint64_t *R_out);
+
 /* Horvitz-Thompson sparse attention for `nrows` query rows (bf16, [nrows][d])
  * of one (b,h) over the tokens of the listed 4-token blocks (ascending), with
  * logit l_t = scale*(q.k_t) - log_pi[block of t]:
@@ -136,6 +154,13 @@ int oracle_sample_plan(int B, int H, int nqb, int nkb, int64_t n,
                        uint64_t seed, const float *scores, int cap,
                        int32_t *counts, int32_t *kv_index, float *log_pi,
                        uint64_t *r_R);
+
+/* oracle_sample_plan with the design chosen: systematic = 0 Poisson,
+ * 1 systematic (oracle_sample_row_systematic). */
+int oracle_sample_plan_design(int B, int H, int nqb, int nkb, int64_t n,
+                              uint64_t seed, const float *scores, int cap,
+                              int32_t *counts, int32_t *kv_index, float *log_pi,
+                              uint64_t *r_R, int systematic);
 
 /* HT sparse attention for every valid query row of query blocks
  * qb_lo <= qb < qb_hi with the given plan.  o is [B,H,N,d] fp64; rows

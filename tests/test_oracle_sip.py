@@ -170,3 +170,85 @@ def test_plan_capacity_formula():
     assert oracle.plan_capacity(8190, 8190) == 8190
     assert oracle.plan_capacity(1512, 18900) == 1856   # 1512 + ceil(311.07) + 32
     assert oracle.plan_capacity(2376, 29700) == 2816   # 2376 + 390 + 32 = 2798 -> 2816
+
+
+# ---------------------------------------------------------------- systematic design
+# The fixed-size alternative (the SIP paragraph fixes the inclusion
+# probabilities, not the design): systematic sampling with probabilities pi.
+# Pins: exactly n blocks in every row, capped blocks always taken, the
+# inclusion probability over the uniform U equal to pi_j (counted on a grid of
+# U values), and agreement with a second formulation written with exact
+# rationals (cumulative pi and the points u, u+1, ..., u+n-1).
+
+def _systematic_by_fractions(s, n, U):
+    from fractions import Fraction
+
+    capped, r, R, _ = oracle.pi_solve(s, n)
+    q = oracle.quantised_scores(s)
+    u = Fraction(U, 1 << 32)
+    take, cum = [], Fraction(0)
+    for qj, c in zip(q, capped):
+        lo = cum
+        cum = cum + (1 if c else Fraction(r * qj, R))
+        # points u + k, k = 0..n-1, below x: max(0, ceil(x - u)) (capped at n)
+        below = lambda x: min(n, max(0, math.ceil(x - u)))
+        take.append(below(cum) > below(lo))
+    assert cum == n
+    return np.array(take)
+
+
+@pytest.mark.parametrize("seed,nkb,n", [(0, 128, 13), (1, 500, 40), (2, 8190, 819), (3, 64, 63),
+                                        (4, 64, 1), (5, 1000, 400), (6, 2000, 7)])
+def test_systematic_takes_exactly_n_including_every_capped_block(seed, nkb, n):
+    s = synthetic.random_scores(1, nkb, seed, concentration=0.3)[0]
+    capped, r, R, _ = oracle.pi_solve(s, n)
+    rng = np.random.default_rng(seed)
+    for U in [0, 1, (1 << 32) - 1] + rng.integers(0, 1 << 32, 5).tolist():
+        take, r2, R2 = oracle.systematic_take(s, n, U)
+        assert (r2, R2) == (r, R)
+        assert int(take.sum()) == n
+        assert bool(take[capped].all())
+
+
+@pytest.mark.parametrize("seed,nkb,n", [(0, 12, 4), (1, 40, 9), (2, 16, 15), (3, 30, 1)])
+def test_systematic_inclusion_probability_is_pi(seed, nkb, n):
+    # over U on a grid of 4096 equally spaced values the block j is taken for
+    # a set of U that is one interval or two (wrapping), of measure pi_j
+    s = synthetic.random_scores(1, nkb, seed, concentration=0.5)[0]
+    p, capped, r, R, q = pis(s, n)
+    grid = [(i << 20) + (1 << 19) for i in range(4096)]
+    counts = np.zeros(nkb)
+    for U in grid:
+        counts += oracle.systematic_take(s, n, U)[0]
+    assert np.all(np.abs(counts - 4096 * np.array(p)) <= 2.0), (counts, p)
+
+
+@pytest.mark.parametrize("seed,nkb,n", [(0, 12, 4), (1, 60, 9), (2, 33, 32), (3, 200, 17)])
+def test_systematic_matches_the_rational_formulation(seed, nkb, n):
+    s = synthetic.random_scores(1, nkb, seed, concentration=0.4)[0]
+    rng = np.random.default_rng(100 + seed)
+    for U in [0, (1 << 32) - 1] + rng.integers(0, 1 << 32, 20).tolist():
+        got, _, _ = oracle.systematic_take(s, n, U)
+        assert np.array_equal(got, _systematic_by_fractions(s, n, U)), U
+
+
+def test_systematic_plan_row_and_layer():
+    s = synthetic.random_scores(3, 300, 8, concentration=0.3)
+    n, cap, seed = 20, oracle.plan_capacity(20, 300), 11
+    for row in range(3):
+        idx, lp, taken, r, R = oracle.sample_row(s[row], n, seed, row, cap, design="systematic")
+        U = oracle.draw_u32(seed, row * 300)
+        take, _, _ = oracle.systematic_take(s[row], n, U)
+        assert taken == n and np.array_equal(idx, np.nonzero(take)[0])
+        capped, r2, R2, _ = oracle.pi_solve(s[row], n)
+        q = oracle.quantised_scores(s[row])
+        for j, l in zip(idx, lp):
+            want = 0.0 if capped[j] else np.float32(math.log(r * q[j] / R))
+            assert l == want
+    plan = oracle.sample_plan(s.reshape(1, 1, 3, 300), n, seed, cap, design="systematic")
+    assert np.all(plan["counts"] == n) and plan["overflow_rows"] == 0
+    idx1, _, _, _, _ = oracle.sample_row(s[1], n, seed, 1, cap, design="systematic")
+    assert np.array_equal(plan["kv_index"][0, 0, 1, :n], idx1)
+    # n >= nkb: every block
+    idx, lp, taken, r, R = oracle.sample_row(s[0], 300, seed, 0, 300, design="systematic")
+    assert taken == 300 and np.array_equal(idx, np.arange(300)) and not lp.any()
