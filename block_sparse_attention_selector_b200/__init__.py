@@ -29,9 +29,14 @@ def version():
     return _abi.version()
 
 
+SAMPLING = {"poisson": _abi.ABSA_SAMPLING_POISSON, "systematic": _abi.ABSA_SAMPLING_SYSTEMATIC}
+
+
 def make_params(B, H, N, d, T, Hg, Wg, budget_blocks, seed=0, softmax_scale=None,
-                kmeans_iters=3):
-    """An absa_params block (q_block 128, kv_block 4, 8 clusters)."""
+                kmeans_iters=3, sampling="poisson"):
+    """An absa_params block (q_block 128, kv_block 4, 8 clusters).
+
+    sampling: "poisson" (independent draws) or "systematic" (exactly budget_blocks blocks)."""
     p = absa_params()
     p.B, p.H, p.N, p.d = int(B), int(H), int(N), int(d)
     p.T, p.Hg, p.Wg = int(T), int(Hg), int(Wg)
@@ -40,12 +45,13 @@ def make_params(B, H, N, d, T, Hg, Wg, budget_blocks, seed=0, softmax_scale=None
     p.budget_blocks = int(budget_blocks)
     p.seed = int(seed) & 0xFFFFFFFFFFFFFFFF
     p.softmax_scale = float(1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale)
+    p.sampling = SAMPLING[sampling]
     return p
 
 
-def params_for(w: Workload, seed=0, budget=None):
+def params_for(w: Workload, seed=0, budget=None, sampling="poisson"):
     return make_params(w.B, w.H, w.N, w.d, w.T, w.Hg, w.Wg,
-                       w.budget if budget is None else budget, seed)
+                       w.budget if budget is None else budget, seed, sampling=sampling)
 
 
 def _stream_handle(stream):

@@ -31,6 +31,8 @@ EXPORTED = (
 )
 
 ABSA_STATIC_SCRATCH_BYTES = 64 << 20
+ABSA_SAMPLING_POISSON = 0
+ABSA_SAMPLING_SYSTEMATIC = 1
 
 
 class absa_params(ctypes.Structure):
@@ -40,7 +42,7 @@ class absa_params(ctypes.Structure):
         ("q_block", ctypes.c_int32), ("kv_block", ctypes.c_int32),
         ("n_clusters", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
         ("budget_blocks", ctypes.c_int32), ("seed", ctypes.c_uint64),
-        ("softmax_scale", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float), ("sampling", ctypes.c_int32),
     ]
 
 

@@ -27,6 +27,7 @@ cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_l
 
 // K4: SIP plan rows from a score array.
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
+                          bool systematic,
                           int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
                           uint64_t *r_R, int32_t *status, int64_t row0, cudaStream_t stream);
 

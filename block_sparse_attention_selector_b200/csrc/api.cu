@@ -133,6 +133,8 @@ absa_status absa_check_params(const absa_params *p) {
     if (p->budget_blocks < 1 || p->kmeans_iters < 1 || p->kmeans_iters > 16)
         return ABSA_ERR_INVALID_ARG;
     if (!isfinite(p->softmax_scale)) return ABSA_ERR_INVALID_ARG;
+    if (p->sampling != ABSA_SAMPLING_POISSON && p->sampling != ABSA_SAMPLING_SYSTEMATIC)
+        return ABSA_ERR_INVALID_ARG;
     if (p->q_block != 128 || p->kv_block != 4 || p->n_clusters != 8) return ABSA_ERR_UNSUPPORTED;
     if (p->d != 64 && p->d != 128) return ABSA_ERR_UNSUPPORTED;
     const Dims dm = dims_of(p);
@@ -215,7 +217,9 @@ absa_status sample_plan_run(const absa_params *p, const float *scores, const abs
     const Dims dm = dims_of(p);
     const int64_t row0 = hr.bh0 * dm.nqb, cap = plan->capacity;
     return from_cuda(launch_sample(scores + row0 * dm.nkb, hr.nbh * dm.nqb, dm.nkb,
-                                   p->budget_blocks, p->seed, plan->capacity, plan->counts + row0,
+                                   p->budget_blocks, p->seed,
+                                   p->sampling == ABSA_SAMPLING_SYSTEMATIC, plan->capacity,
+                                   plan->counts + row0,
                                    plan->kv_index + row0 * cap, plan->log_pi + row0 * cap,
                                    plan->r_R + 2 * row0, plan->status, row0, s));
 }

@@ -1,8 +1,10 @@
 // sample.cu -- SIP sampler on sm_100a (AB-Attention summary page, "AB-Attention's
 // three techniques", SIP paragraph): inclusion probability proportional to the
 // block score, the top blocks capped at pi = 1, the rest keeping a nonzero
-// chance, sum pi = budget; independent (Poisson) draws from a counter-based
-// hash; ascending compaction of the taken blocks with their ln(pi).
+// chance, sum pi = budget; draws from a counter-based hash, either
+// independent per block (Poisson design) or one per row for systematic
+// sampling (exactly `budget` blocks; the paragraph fixes the probabilities,
+// not the design); ascending compaction of the taken blocks with their ln(pi).
 //
 // Integer formulation (exact, so every ordering of the reductions gives the
 // same plan): q_j = max(1, floor(s_j 2^32)); capping fixed point on
@@ -43,6 +45,15 @@ constexpr int kCandMax = 2048;
 // comparison reduces to u Rh + hi32(u Rl) < rq.
 __device__ __forceinline__ bool draw_taken(uint32_t u, uint32_t Rh, uint32_t Rl, uint64_t rq) {
     return (uint64_t)u * Rh + __umulhi(u, Rl) < rq;
+}
+
+// (x + y) mod R and (x - y) mod R for x, y < R < 2^49.
+__device__ __forceinline__ uint64_t addmod(uint64_t x, uint64_t y, uint64_t R) {
+    const uint64_t z = x + y;
+    return z >= R ? z - R : z;
+}
+__device__ __forceinline__ uint64_t submod(uint64_t x, uint64_t y, uint64_t R) {
+    return x >= y ? x - y : x + R - y;
 }
 
 constexpr int kSampleThreads = 256;
@@ -89,7 +100,7 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
 __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
-    uint64_t *__restrict__ r_R, int32_t *status, int64_t row0) {
+    uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, bool systematic) {
     extern __shared__ __align__(16) uint32_t samp_smem[];
     const int ngroups = (nkb + 31) >> 5;
     uint32_t *qm1 = samp_smem;                      // [ngroups*32]
@@ -261,27 +272,72 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     }
     const uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
 
-    // Poisson draws: one taken word per group; SplitMix64 state of block j is
-    // base + j * gamma with base = mix(seed) + (global row * NKB + 1) * gamma
+    // SplitMix64 state of block j is base + j * gamma with
+    // base = mix(seed) + (global row * NKB + 1) * gamma
     const uint64_t base =
         splitmix64_mix(seed) + ((uint64_t)(row0 + row) * (uint64_t)nkb + 1) * kGamma;
     const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
     int taken = 0;
-    uint64_t state = base + (uint64_t)(g0 * 32 + lane) * kGamma;  // state of block j
-    for (int g = g0; g < g1; ++g, state += 32 * kGamma) {
-        const int j = g * 32 + lane;
-        bool take = false;
-        if (j < nkb) {
-            if ((capw[g] >> lane) & 1u) {
-                take = true;
-            } else {
-                const uint64_t rq = (uint64_t)r32 * qm1[j] + r32;
-                take = draw_taken(splitmix64_hi32(state), Rh, Rl, rq);
+    if (!systematic) {
+        // Poisson draws: one taken word per group
+        uint64_t state = base + (uint64_t)(g0 * 32 + lane) * kGamma;  // state of block j
+        for (int g = g0; g < g1; ++g, state += 32 * kGamma) {
+            const int j = g * 32 + lane;
+            bool take = false;
+            if (j < nkb) {
+                if ((capw[g] >> lane) & 1u) {
+                    take = true;
+                } else {
+                    const uint64_t rq = (uint64_t)r32 * qm1[j] + r32;
+                    take = draw_taken(splitmix64_hi32(state), Rh, Rl, rq);
+                }
             }
+            const uint32_t tw = __ballot_sync(0xffffffffu, take);
+            if (lane == 0) takew[g] = tw;
+            taken += __popc(tw);
         }
-        const uint32_t tw = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) takew[g] = tw;
-        taken += __popc(tw);
+    } else {
+        // Systematic design.  Interval j is [A_j, A_j + a_j) with a_j = R on C
+        // and r q_j elsewhere, A_j = sum_{i<j} a_i; the points are
+        // (k + U/2^32) R.  With rho_j = A_j mod R (capped blocks add 0 mod R)
+        // and F = floor(U R / 2^32), an uncapped interval (a_j < R) holds the
+        // point of its own period iff rho_j <= F < rho_j + a_j and that of
+        // the next period iff R + F < rho_j + a_j (comparisons of the exact
+        // values U R vs multiples of 2^32 reduce to these on F).
+        const uint32_t U = splitmix64_hi32(base);  // the draw of block 0 of the row
+        const uint64_t F = (uint64_t)U * Rh + __umulhi(U, Rl);
+        // warp totals of a_j mod R, then this warp's starting rho
+        uint64_t tot = 0;
+        for (int g = g0; g < g1; ++g) {
+            const int j = g * 32 + lane;
+            if (j < nkb && !((capw[g] >> lane) & 1u))
+                tot = addmod(tot, (uint64_t)r32 * qm1[j] + r32, R);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tot = addmod(tot, __shfl_xor_sync(0xffffffffu, tot, o), R);
+        __syncthreads();  // earlier readers of red_a are done
+        if (lane == 0) red_a[warp] = tot;
+        __syncthreads();
+        uint64_t carry = 0;
+        for (int w = 0; w < warp; ++w) carry = addmod(carry, red_a[w], R);
+        for (int g = g0; g < g1; ++g) {
+            const int j = g * 32 + lane;
+            const bool cp = (capw[g] >> lane) & 1u;
+            const uint64_t a = (j < nkb && !cp) ? (uint64_t)r32 * qm1[j] + r32 : 0;
+            uint64_t inc = a;  // inclusive scan over the group, mod R
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc = addmod(inc, y, R);
+            }
+            const uint64_t rho = addmod(carry, submod(inc, a, R), R);
+            bool take = false;
+            if (j < nkb) take = cp || (rho <= F && F < rho + a) || (R + F < rho + a);
+            carry = addmod(carry, __shfl_sync(0xffffffffu, inc, 31), R);
+            const uint32_t tw = __ballot_sync(0xffffffffu, take);
+            if (lane == 0) takew[g] = tw;
+            taken += __popc(tw);
+        }
     }
     if (lane == 0) warp_cnt[warp] = taken;
     __syncthreads();
@@ -327,15 +383,16 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
 }
 
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
-                          int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
-                          uint64_t *r_R, int32_t *status, int64_t row0, cudaStream_t stream) {
+                          bool systematic, int cap, int32_t *counts, int32_t *kv_index,
+                          float *log_pi, uint64_t *r_R, int32_t *status, int64_t row0,
+                          cudaStream_t stream) {
     const int ngroups = (nkb + 31) / 32;
     const int smem = (ngroups * 32 + 2 * ngroups + kCandMax) * 4;
     cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     absa_sample_kernel<<<(unsigned)rows, kSampleThreads, smem, stream>>>(
-        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0);
+        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0, systematic);
     return cudaGetLastError();
 }
 

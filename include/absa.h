@@ -64,7 +64,13 @@ typedef struct {
     int32_t budget_blocks;  /* n: expected KV blocks per query block; n >= NKB = dense */
     uint64_t seed;          /* SIP draw seed                                          */
     float softmax_scale;    /* logit scale, normally 1/sqrt(d)                        */
+    int32_t sampling;       /* SIP design: ABSA_SAMPLING_POISSON (0, the default) or  */
+                            /* ABSA_SAMPLING_SYSTEMATIC (1); see absa_sample_plan     */
 } absa_params;
+
+/* Sampling designs of the SIP sampler (absa_params.sampling). */
+#define ABSA_SAMPLING_POISSON 0
+#define ABSA_SAMPLING_SYSTEMATIC 1
 
 typedef struct {
     /* All arrays are caller-owned device memory sized from absa_plan_capacity. */
@@ -123,11 +129,19 @@ absa_status absa_select_scores(const absa_params *p, const void *q, const void *
  * Integer inclusion probabilities: q_j = max(1, floor(s_j * 2^32)) (NaN or
  * negative -> 1, at most 2^32); from C = {} repeat r = n - |C|,
  * R = sum_{j not in C} q_j, C += {j : r*q_j >= R} until C is unchanged;
- * pi_j = 1 on C, r*q_j/R elsewhere, so sum pi = n exactly.  Poisson draws:
- * with ctr = row*NKB + j, row = (b*H + h)*NQB + qb, and mix the SplitMix64
- * output function, u_j = mix(mix(seed) + (ctr+1)*0x9E3779B97F4A7C15) >> 32
- * (output ctr+1 of SplitMix64 started from state mix(seed)); block j is taken
- * iff j in C or u_j * R < r*q_j * 2^32.  Taken blocks are written ascending
+ * pi_j = 1 on C, r*q_j/R elsewhere, so sum pi = n exactly.  Draws: with
+ * ctr = row*NKB + j, row = (b*H + h)*NQB + qb, and mix the SplitMix64 output
+ * function, u(ctr) = mix(mix(seed) + (ctr+1)*0x9E3779B97F4A7C15) >> 32
+ * (output ctr+1 of SplitMix64 started from state mix(seed)).
+ *  - ABSA_SAMPLING_POISSON: block j is taken iff j in C or
+ *    u(row*NKB + j) * R < r*q_j * 2^32 (independent draws; the sample size
+ *    is random with mean n).
+ *  - ABSA_SAMPLING_SYSTEMATIC: the blocks are laid end to end in ascending j
+ *    with lengths a_j = R on C and r*q_j elsewhere (sum n*R); with
+ *    U = u(row*NKB), points sit at (k + U/2^32)*R for k = 0..n-1 and block j
+ *    is taken iff a point falls in [sum_{i<j} a_i, sum_{i<=j} a_i).  Every
+ *    block is taken with probability pi_j and exactly n blocks are taken.
+ * Taken blocks are written ascending
  * with log_pi = 0 (capped) or (float)ln((double)(r*q_j)/R).  n >= NKB takes
  * every block.  Resets plan->status first; a row with more than
  * plan->capacity blocks keeps the first `capacity` and sets

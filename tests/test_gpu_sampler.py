@@ -14,14 +14,15 @@ from gpu_helpers import plan_to_numpy
 pytestmark = pytest.mark.gpu
 
 
-def _params(nkb, rows_h, n, seed):
+def _params(nkb, rows_h, n, seed, sampling="poisson"):
     # a one-row-per-head layout: B=1, H=rows_h, N=4*nkb tokens with NQB = ceil(4 nkb / 128)
     N = 4 * nkb
-    return make_params(1, rows_h, N, 128, 1, 1, N, n, seed=seed)
+    return make_params(1, rows_h, N, 128, 1, 1, N, n, seed=seed, sampling=sampling)
 
 
 def _compare(p, scores, plan_gpu, cap):
-    ref = oracle.sample_plan(scores, p.budget_blocks, p.seed, cap)
+    design = "systematic" if p.sampling == _abi.ABSA_SAMPLING_SYSTEMATIC else "poisson"
+    ref = oracle.sample_plan(scores, p.budget_blocks, p.seed, cap, design=design)
     got = plan_to_numpy(plan_gpu)
     assert np.array_equal(got["counts"], ref["counts"])
     assert np.array_equal(got["r_R"], ref["r_R"])
@@ -102,3 +103,56 @@ def test_sampler_full_wan480_rows():
     plan = sample_plan(p, torch.from_numpy(scores).cuda())
     plan.check()
     _compare(p, scores, plan, plan.capacity)
+
+
+# The systematic design (exactly n blocks per row): same bar, every row of
+# exactly n entries.
+@pytest.mark.parametrize("nkb,H,n,seed,conc", [(128, 2, 13, 0, 3.0), (1000, 3, 100, 1, 0.3),
+                                               (8190, 2, 819, 2, 3.0), (29700, 1, 2376, 3, 3.0),
+                                               (515, 2, 1, 4, 3.0), (515, 2, 514, 5, 3.0),
+                                               (8190, 1, 82, 6, 0.2), (18900, 1, 1512, 7, 1.0)])
+def test_systematic_sampler_bit_exact_on_identical_scores(nkb, H, n, seed, conc):
+    import torch
+
+    p = _params(nkb, H, n, seed, sampling="systematic")
+    nqb = (p.N + 127) // 128
+    scores = synthetic.random_scores(H * nqb, nkb, seed, concentration=conc).reshape(1, H, nqb,
+                                                                                     nkb)
+    plan = sample_plan(p, torch.from_numpy(scores).cuda())
+    plan.check()
+    ref = _compare(p, scores, plan, plan.capacity)
+    assert np.all(ref["counts"] == n)
+
+
+def test_systematic_full_layer_plan_and_attention():
+    """select_plan with the systematic design on the Wan2.1 480p layer cut to 4
+    heads: exactly n blocks per row, the plan bit-equal to the oracle's from
+    the GPU's own scores, and sparse attention on it against the oracle on
+    sampled query blocks."""
+    import dataclasses
+    import math
+
+    import torch
+    from block_sparse_attention_selector_b200 import params_for, select_plan, sparse_attention
+    from gpu_helpers import ATTN_MAX_ABS, ATTN_REL_L2, attention_errors, device_bf16
+
+    w = dataclasses.replace(synthetic.WAN480, H=4)
+    q, k, v = synthetic.layer_qkv_bits(w)
+    p = params_for(w, seed=9, sampling="systematic")
+    qd, kd, vd = device_bf16(q), device_bf16(k), device_bf16(v)
+    plan, scores, _ = select_plan(p, qd, kd)
+    o = sparse_attention(p, qd, kd, vd, plan)
+    plan.check()
+    assert bool((plan.counts == w.budget).all())
+    s = scores.cpu().numpy()
+    ref = _compare(p, s, plan, plan.capacity)
+    for h in (0, w.H - 1):
+        for qb in (0, w.nqb // 2, w.nqb - 1):
+            m = min(128, w.N - 128 * qb)
+            rows = slice(128 * qb, 128 * qb + m)
+            c = int(ref["counts"][0, h, qb])
+            o_ref = oracle.sparse_attention_rows(q[0, h, rows], k[0, h], v[0, h],
+                                                 ref["kv_index"][0, h, qb, :c],
+                                                 ref["log_pi"][0, h, qb, :c], 1 / math.sqrt(w.d))
+            mx, rel = attention_errors(o[0, h, rows].float().cpu().numpy(), o_ref)
+            assert mx <= ATTN_MAX_ABS and rel <= ATTN_REL_L2, (h, qb, mx, rel)
