@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads (profiling captures); 0 = all 40")
     ap.add_argument("--dense-reps", type=int, default=3)
+    ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic"],
+                    help="SIP design: Poisson draws (default) or systematic (exactly n blocks)")
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep and 16-step plan-reuse schedule (JSON lines; no main line)")
     return ap.parse_args()
@@ -63,9 +65,10 @@ def workload(heads=0):
     return w
 
 
-def config_of(w, extra=None):
+def config_of(w, extra=None, sampling="poisson"):
     cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-           "grid": [w.T, w.Hg, w.Wg], "budget_blocks": w.budget, "kv_blocks": w.nkb,
+           "grid": [w.T, w.Hg, w.Wg], "budget_blocks": w.budget, "sampling": sampling,
+           "kv_blocks": w.nkb,
            "query_blocks": w.nqb, "inputs": "seeded synthetic Fourier-feature q/k, Gaussian v",
            "l2": "flushed before every timed step (256 MiB write, outside the step events); "
                  "inputs (1 GiB q/k/v) are also larger than L2"}
@@ -76,7 +79,7 @@ def config_of(w, extra=None):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_sample(w, q, k, v, n_qb, seed=1):
+def oracle_sample(w, q, k, v, n_qb, seed=1, design="poisson"):
     """Run the oracle hot path on query blocks [0, n_qb) of every head; seconds."""
     import oracle
 
@@ -84,7 +87,7 @@ def oracle_sample(w, q, k, v, n_qb, seed=1):
     scores, _, _, _ = oracle.select_scores(q, k, qb_range=(0, n_qb))
     sub = np.ascontiguousarray(scores[:, :, :n_qb])
     cap = oracle.plan_capacity(w.budget, w.nkb)
-    plan = oracle.sample_plan(sub, w.budget, seed, cap)
+    plan = oracle.sample_plan(sub, w.budget, seed, cap, design=design)
     full = dict(counts=np.zeros((w.B, w.H, w.nqb), np.int32),
                 kv_index=np.zeros((w.B, w.H, w.nqb, cap), np.int32),
                 log_pi=np.zeros((w.B, w.H, w.nqb, cap), np.float32))
@@ -95,12 +98,12 @@ def oracle_sample(w, q, k, v, n_qb, seed=1):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, q, k, v, target_s):
+def cpu_baseline(w, q, k, v, target_s, design="poisson"):
     import oracle
 
-    t1 = oracle_sample(w, q, k, v, 1)
+    t1 = oracle_sample(w, q, k, v, 1, design=design)
     n_qb = int(max(1, min(w.nqb, math.floor(target_s / max(t1, 1e-3)))))
-    t = oracle_sample(w, q, k, v, n_qb) if n_qb > 1 else t1
+    t = oracle_sample(w, q, k, v, n_qb, design=design) if n_qb > 1 else t1
     ms = t * 1e3 * w.nqb / n_qb
     return {"value": ms, "unit": "ms", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"query blocks 0..{n_qb - 1} of all {w.H} heads ({n_qb * w.H} of "
@@ -121,18 +124,18 @@ def run_reference(args):
     oracle.lib()
     steps = max(1, args.steps)
     per_step_target = max(1.0, min(args.cpu_seconds, 120.0 / (steps + args.warmup)))
-    t1 = oracle_sample(w, q, k, v, 1)
+    t1 = oracle_sample(w, q, k, v, 1, design=args.sampling)
     n_qb = int(max(1, min(w.nqb, math.floor(per_step_target / max(t1, 1e-3)))))
     for _ in range(args.warmup):
-        oracle_sample(w, q, k, v, n_qb)
-    times = [oracle_sample(w, q, k, v, n_qb) for _ in range(steps)]
+        oracle_sample(w, q, k, v, n_qb, design=args.sampling)
+    times = [oracle_sample(w, q, k, v, n_qb, design=args.sampling) for _ in range(steps)]
     ms = float(np.mean(times)) * 1e3 * w.nqb / n_qb
     sample = (f"each step: query blocks 0..{n_qb - 1} of all {w.H} heads "
               f"(select+sample+attention), extrapolated x{w.nqb / n_qb:.1f}")
     line = {"impl": "reference", "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w),
+            "config": config_of(w, sampling=args.sampling),
             "cpu_baseline": {"value": ms, "unit": "ms", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -247,7 +250,7 @@ def run_ours(args):
         return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
 
     q, k, v = to_dev(q_bits), to_dev(k_bits), to_dev(v_bits)
-    p = absa.params_for(w, seed=1234 + rank)
+    p = absa.params_for(w, seed=1234 + rank, sampling=args.sampling)
     plan = absa.Plan(p, dev)
     scores = torch.empty((w.B, w.H, w.nqb, w.nkb), dtype=torch.float32, device=dev)
     ws = absa.workspace(p, dev)
@@ -371,7 +374,7 @@ def run_ours(args):
                                  / 1e12) if dense_ms else None,
                 "mean_blocks_per_row": float(counts.mean()),
                 "selector_hbm_frac_of_measured": sel_bytes / (float(sel.mean()) * 1e-3) / 1e9 / hbm_gbs,
-            }),
+            }, sampling=args.sampling),
             "roofline": {"bound": "tensor", "kernel": "absa_attention_kernel<128,sparse>",
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": achieved_tf / peak_tf,
@@ -392,7 +395,8 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(w, q_bits, k_bits, v_bits, args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(w, q_bits, k_bits, v_bits, args.cpu_seconds,
+                                                design=args.sampling)
         print(json.dumps(line), flush=True)
     return 0
 
@@ -440,10 +444,10 @@ def run_sweep(args):
         o_dense, dense_ms = timed(lambda: absa.dense_reference(p0, q, k, v))
     dense_rms = float(o_dense.float().pow(2).mean().sqrt())
     v_rms = float(v.float().pow(2).mean().sqrt())
-    for budget in SWEEP_BUDGETS:
+    for budget, design in [(b, d) for b in SWEEP_BUDGETS for d in ("poisson", "systematic")]:
         sel, att, rel, blocks = [], [], [], []
         for seed in range(8):
-            p = absa.params_for(w, seed=seed, budget=budget)
+            p = absa.params_for(w, seed=seed, budget=budget, sampling=design)
             (plan, _, _), t_sel = timed(lambda: absa.select_plan(p, q, k))
             plan.check()
             for _ in range(4):  # one plan, four attention calls
@@ -453,6 +457,7 @@ def run_sweep(args):
             rel.append(rel_l2(o, o_dense))
             blocks.append(float(plan.counts.float().mean()))
         line = {"kind": "density_sweep", "workload": w.name, "budget_blocks": budget,
+                "sampling": design,
                 "density": budget / w.nkb, "mean_blocks_per_row": float(np.mean(blocks)),
                 "select_plan_ms": float(np.median(sel)), "attention_ms": float(np.median(att)),
                 "ms_per_call_plan_reused_4x": float(np.median(sel)) / 4 + float(np.median(att)),

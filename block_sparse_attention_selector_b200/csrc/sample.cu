@@ -103,10 +103,12 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, bool systematic) {
     extern __shared__ __align__(16) uint32_t samp_smem[];
     const int ngroups = (nkb + 31) >> 5;
-    uint32_t *qm1 = samp_smem;                      // [ngroups*32]
-    uint32_t *capw = samp_smem + ngroups * 32;      // [ngroups]
-    uint32_t *takew = capw + ngroups;               // [ngroups]
-    uint32_t *cand = takew + ngroups;               // [kCandMax]
+    const int ngp = (ngroups + 7) & ~7;             // groups rounded up to whole 256-block
+                                                    // super-groups (systematic pass)
+    uint32_t *qm1 = samp_smem;                      // [ngp*32]
+    uint32_t *capw = samp_smem + ngp * 32;          // [ngp]
+    uint32_t *takew = capw + ngp;                   // [ngp]
+    uint32_t *cand = takew + ngp;                   // [kCandMax]
     __shared__ uint64_t red_a[kSampleWarps];
     __shared__ int red_b[kSampleWarps];
     __shared__ int warp_cnt[kSampleWarps];
@@ -304,40 +306,71 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         // point of its own period iff rho_j <= F < rho_j + a_j and that of
         // the next period iff R + F < rho_j + a_j (comparisons of the exact
         // values U R vs multiples of 2^32 reduce to these on F).
+        // Blocks go in super-groups of 256: lane l holds the 8 consecutive
+        // blocks 8l..8l+7, sums them in order and one warp scan per
+        // super-group gives each lane its starting rho; the 8 taken bits are
+        // the lane's byte of the group's taken word.
         const uint32_t U = splitmix64_hi32(base);  // the draw of block 0 of the row
         const uint64_t F = (uint64_t)U * Rh + __umulhi(U, Rl);
-        // warp totals of a_j mod R, then this warp's starting rho
+        const int nsg = ngp >> 3;
+        const int sg_per_warp = (nsg + kSampleWarps - 1) / kSampleWarps;
+        const int s0 = warp * sg_per_warp, s1 = min(nsg, s0 + sg_per_warp);
+        // a_j mod R of the lane's 8 blocks (0 when capped or past NKB) and their capped bits
+        auto elems = [&](int sg, uint64_t (&e)[8], uint32_t &cb) {
+            const int j0 = sg * 256 + lane * 8;
+            const uint4 v0 = *reinterpret_cast<const uint4 *>(qm1 + j0);
+            const uint4 v1 = *reinterpret_cast<const uint4 *>(qm1 + j0 + 4);
+            const uint32_t qv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const int valid = min(8, max(0, nkb - j0));
+            cb = (capw[j0 >> 5] >> (j0 & 31)) & ((1u << valid) - 1u);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                e[i] = (i < valid && !((cb >> i) & 1u)) ? (uint64_t)r32 * qv[i] + r32 : 0;
+        };
         uint64_t tot = 0;
-        for (int g = g0; g < g1; ++g) {
-            const int j = g * 32 + lane;
-            if (j < nkb && !((capw[g] >> lane) & 1u))
-                tot = addmod(tot, (uint64_t)r32 * qm1[j] + r32, R);
+        for (int sg = s0; sg < s1; ++sg) {
+            uint64_t e[8];
+            uint32_t cb;
+            elems(sg, e, cb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tot = addmod(tot, e[i], R);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) tot = addmod(tot, __shfl_xor_sync(0xffffffffu, tot, o), R);
         __syncthreads();  // earlier readers of red_a are done
         if (lane == 0) red_a[warp] = tot;
         __syncthreads();
-        uint64_t carry = 0;
+        uint64_t carry = 0;  // rho of this warp's first block
         for (int w = 0; w < warp; ++w) carry = addmod(carry, red_a[w], R);
-        for (int g = g0; g < g1; ++g) {
-            const int j = g * 32 + lane;
-            const bool cp = (capw[g] >> lane) & 1u;
-            const uint64_t a = (j < nkb && !cp) ? (uint64_t)r32 * qm1[j] + r32 : 0;
-            uint64_t inc = a;  // inclusive scan over the group, mod R
+        uint8_t *takeb = reinterpret_cast<uint8_t *>(takew);
+        for (int sg = s0; sg < s1; ++sg) {
+            uint64_t e[8];
+            uint32_t cb;
+            elems(sg, e, cb);
+            uint64_t lt = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lt = addmod(lt, e[i], R);
+            uint64_t inc = lt;  // inclusive scan of the lane totals, mod R
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc = addmod(inc, y, R);
             }
-            const uint64_t rho = addmod(carry, submod(inc, a, R), R);
-            bool take = false;
-            if (j < nkb) take = cp || (rho <= F && F < rho + a) || (R + F < rho + a);
+            uint64_t rho = addmod(carry, submod(inc, lt, R), R);
+            uint32_t bits = cb;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint64_t a = e[i];
+                if (a != 0 && ((rho <= F && F < rho + a) || R + F < rho + a)) bits |= 1u << i;
+                rho = addmod(rho, a, R);
+            }
+            takeb[sg * 32 + lane] = (uint8_t)bits;  // byte lane&3 of group word sg*8 + lane/4
             carry = addmod(carry, __shfl_sync(0xffffffffu, inc, 31), R);
-            const uint32_t tw = __ballot_sync(0xffffffffu, take);
-            if (lane == 0) takew[g] = tw;
-            taken += __popc(tw);
         }
+        __syncthreads();  // taken words written by other warps
+        for (int g = g0 + lane; g < g1; g += 32) taken += __popc(takew[g]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) taken += __shfl_xor_sync(0xffffffffu, taken, o);
     }
     if (lane == 0) warp_cnt[warp] = taken;
     __syncthreads();
@@ -387,7 +420,8 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
                           float *log_pi, uint64_t *r_R, int32_t *status, int64_t row0,
                           cudaStream_t stream) {
     const int ngroups = (nkb + 31) / 32;
-    const int smem = (ngroups * 32 + 2 * ngroups + kCandMax) * 4;
+    const int ngp = (ngroups + 7) & ~7;
+    const int smem = (ngp * 32 + 2 * ngp + kCandMax) * 4;
     cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
