@@ -193,8 +193,8 @@ class ClockSampler:
                 for name, val in zip(names, parts[5:9]):
                     if val.lower() == "active":
                         reasons.add(name)
-        if not sm:
-            return None
+        if not sm:  # timed region shorter than the sampling period
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
 
@@ -350,7 +350,7 @@ def run_ours(args):
     # The timed region is a loop of K steps; once it runs long enough for the
     # power cap to act (or the sampler saw it act) the matching denominator is
     # the sustained GEMM figure, otherwise the burst one.
-    long_loop = float(tot.sum()) >= 500.0 or "sw_power_cap" in clk.get("reasons", [])
+    long_loop = float(tot.sum()) >= 500.0 or "sw_power_cap" in (clk or {}).get("reasons", [])
     peak_tf = sustained_tf if long_loop else burst_tf
     peak_kind = "sustained" if long_loop else "burst"
     att_ms = float(att.mean())
