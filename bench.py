@@ -49,6 +49,12 @@ def parse():
     ap.add_argument("--dense-reps", type=int, default=3)
     ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic"],
                     help="SIP design: Poisson draws (default) or systematic (exactly n blocks)")
+    ap.add_argument("--harness", action="store_true",
+                    help="mass-retention / error harness on the 480p and 720p layers (JSON lines; "
+                         "no main line)")
+    ap.add_argument("--harness-heads", type=int, default=8,
+                    help="heads of the 720p layers in the harness (the 480p layer uses --heads or "
+                         "all 40)")
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep and 16-step plan-reuse schedule (JSON lines; no main line)")
     return ap.parse_args()
@@ -495,12 +501,44 @@ def run_sweep(args):
     return 0
 
 
+def run_harness(args):
+    """Retained attention mass and error vs dense of ideal top-k, block-mean, IBCS top-n and
+    both SIP designs at the layer's budget, plus 128-token ideal top-k at the same key fraction.
+    One JSON line per layer."""
+    import dataclasses
+
+    import torch
+
+    from block_sparse_attention_selector_b200 import harness, synthetic
+
+    dev = torch.device("cuda", 0)
+    layers = [workload(args.heads)]
+    for w in (synthetic.WAN720, synthetic.HUNYUAN720):
+        h = min(w.H, args.harness_heads)
+        layers.append(dataclasses.replace(w, H=h, name=f"{w.name}_{h}heads") if h < w.H else w)
+    for w in layers:
+        q_bits, k_bits, v_bits = synthetic.layer_qkv_bits(w)
+
+        def to_dev(b):
+            return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+        q, k, v = to_dev(q_bits), to_dev(k_bits), to_dev(v_bits)
+        rep, _ = harness.retention_report(w, q, k, v, seed=1)
+        rep["kind"] = "mass_retention"
+        print(json.dumps(rep), flush=True)
+        del q, k, v
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.harness:
+        return run_harness(args)
     return run_ours(args)
 
 
