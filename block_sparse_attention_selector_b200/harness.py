@@ -24,7 +24,6 @@ attention and score computation runs in the library's kernels.
 """
 import math
 
-
 from . import Plan, dense_reference, params_for, sample_plan, select_scores, sparse_attention
 
 
