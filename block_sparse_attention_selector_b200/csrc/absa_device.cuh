@@ -11,6 +11,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -257,6 +258,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
            | ((uint32_t)b_mn_major << 16)    // B major
            | ((uint32_t)(N >> 3) << 17)      // N / 8
            | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+// The same with fp16 A and B (format code 0 for both operands).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int b_mn_major) {
+    return (1u << 4)                         // D format f32
+           | ((uint32_t)b_mn_major << 16)    // B major
+           | ((uint32_t)(N >> 3) << 17)      // N / 8
+           | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+// fp16 of x, round to nearest even, clamped to the finite range (+-65504).
+__device__ __forceinline__ __half f16_sat(float x) {
+    return __float2half_rn(fminf(fmaxf(x, -65504.f), 65504.f));
 }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside an SW128 region.

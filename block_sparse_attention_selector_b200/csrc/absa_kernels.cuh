@@ -9,21 +9,21 @@ namespace absa {
 
 constexpr int kSampleMaxKvBlocks = 49152;
 
-// K1: mean key of every 4-token block as bf16 hi + lo.
-cudaError_t launch_pool(const __nv_bfloat16 *k, __nv_bfloat16 *kbar_hi, __nv_bfloat16 *kbar_lo,
+// K1: mean key of every 4-token block as fp16 hi + lo.
+cudaError_t launch_pool(const __nv_bfloat16 *k, __half *kbar_hi, __half *kbar_lo,
                         int64_t BH, int N, int nkb, int d, cudaStream_t stream);
 
-// K2: per-query-block k-means (8 clusters), centroids, their bf16 split,
+// K2: per-query-block k-means (8 clusters), centroids, their fp16 split,
 // weights and final assignment.
 cudaError_t launch_kmeans(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int d, int iters,
-                          float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
+                          float *mu, __half *mu_hi, __half *mu_lo, float *w,
                           uint8_t *assign, cudaStream_t stream);
 
-// K3: block scores from the centroid split and the key-block split.
+// K3: block scores from the centroids (fp16 hi) and the key-block split (fp16 hi + lo).
 cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,
-                         const CUtensorMap &tm_mu_hi, const CUtensorMap &tm_mu_lo, const float *w,
-                         float *scores, int64_t BH, int nqb, int nkb, int d, float softmax_scale,
-                         int32_t *status, cudaStream_t stream);
+                         const CUtensorMap &tm_mu_hi, const float *w, float *scores, int64_t BH,
+                         int nqb, int nkb, int d, float softmax_scale, int32_t *status,
+                         cudaStream_t stream);
 
 // K4: SIP plan rows from a score array.
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,

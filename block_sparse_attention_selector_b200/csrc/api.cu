@@ -75,19 +75,29 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (cols fastest), box 64 x box_rows with 128-byte swizzle.
-bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int cols,
-                   int box_rows = 128) {
+// 2-D tensor of 16-bit elements [rows, cols] (cols fastest), box 64 x box_rows with
+// 128-byte swizzle.
+bool make_map_16(CUtensorMap *map, const void *base, int64_t rows, int cols, int box_rows,
+                 CUtensorMapDataType dtype) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estride[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), gdim, gstride,
+    return fn(map, dtype, 2, const_cast<void *>(base), gdim, gstride,
               box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int cols,
+                   int box_rows = 128) {
+    return make_map_16(map, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+bool make_map_f16(CUtensorMap *map, const void *base, int64_t rows, int cols) {
+    return make_map_16(map, base, rows, cols, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
 }
 
 absa_status check_plan(const absa_params *p, const absa_plan *plan) {
@@ -184,22 +194,21 @@ absa_status select_scores_run(const absa_params *p, const void *q, const void *k
     const Dims dm = dims_of(p);
     const int64_t d = p->d;
     uint8_t *w8 = static_cast<uint8_t *>(ws);
-    auto *kb_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_hi) + hr.bh0 * dm.nkb * d;
-    auto *kb_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.kbar_lo) + hr.bh0 * dm.nkb * d;
+    auto *kb_hi = reinterpret_cast<__half *>(w8 + L.kbar_hi) + hr.bh0 * dm.nkb * d;
+    auto *kb_lo = reinterpret_cast<__half *>(w8 + L.kbar_lo) + hr.bh0 * dm.nkb * d;
     auto *mu = reinterpret_cast<float *>(w8 + L.mu) + hr.bh0 * dm.nqb * 8 * d;
-    auto *mu_hi = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_hi) + hr.bh0 * dm.nqb * 8 * d;
-    auto *mu_lo = reinterpret_cast<__nv_bfloat16 *>(w8 + L.mu_lo) + hr.bh0 * dm.nqb * 8 * d;
+    auto *mu_hi = reinterpret_cast<__half *>(w8 + L.mu_hi) + hr.bh0 * dm.nqb * 8 * d;
+    auto *mu_lo = reinterpret_cast<__half *>(w8 + L.mu_lo) + hr.bh0 * dm.nqb * 8 * d;
     auto *w = reinterpret_cast<float *>(w8 + L.w) + hr.bh0 * dm.nqb * 8;
     auto *assign = w8 + L.assign + hr.bh0 * dm.nqb * 128;
     const auto *qh = static_cast<const __nv_bfloat16 *>(q) + hr.bh0 * p->N * d;
     const auto *kh = static_cast<const __nv_bfloat16 *>(k) + hr.bh0 * p->N * d;
     float *sh = scores + hr.bh0 * dm.nqb * (int64_t)dm.nkb;
 
-    CUtensorMap tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo;
-    if (!make_map_bf16(&tm_kb_hi, kb_hi, hr.nbh * dm.nkb, p->d) ||
-        !make_map_bf16(&tm_kb_lo, kb_lo, hr.nbh * dm.nkb, p->d) ||
-        !make_map_bf16(&tm_mu_hi, mu_hi, hr.nbh * dm.nqb * 8, p->d) ||
-        !make_map_bf16(&tm_mu_lo, mu_lo, hr.nbh * dm.nqb * 8, p->d))
+    CUtensorMap tm_kb_hi, tm_kb_lo, tm_mu_hi;
+    if (!make_map_f16(&tm_kb_hi, kb_hi, hr.nbh * dm.nkb, p->d) ||
+        !make_map_f16(&tm_kb_lo, kb_lo, hr.nbh * dm.nkb, p->d) ||
+        !make_map_f16(&tm_mu_hi, mu_hi, hr.nbh * dm.nqb * 8, p->d))
         return ABSA_ERR_CUDA;
 
     cudaError_t e = launch_pool(kh, kb_hi, kb_lo, hr.nbh, p->N, dm.nkb, p->d, s);
@@ -207,7 +216,7 @@ absa_status select_scores_run(const absa_params *p, const void *q, const void *k
     e = launch_kmeans(qh, hr.nbh, p->N, dm.nqb, p->d, p->kmeans_iters, mu, mu_hi, mu_lo, w, assign,
                       s);
     if (e != cudaSuccess) return from_cuda(e);
-    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, sh, hr.nbh, dm.nqb, dm.nkb, p->d,
+    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, sh, hr.nbh, dm.nqb, dm.nkb, p->d,
                      p->softmax_scale, status, s);
     return from_cuda(e);
 }

@@ -12,10 +12,11 @@ namespace absa {
 
 // One thread per (row = (b,h,j), 8-element chunk): reads the 4 token rows of
 // block j (16-byte loads, a warp covers whole rows), averages in fp32 and
-// stores mean = hi + lo with hi = bf16(mean), lo = bf16(mean - hi).
+// stores mean = hi + lo with hi = fp16(mean), lo = fp16(mean - hi) (round to
+// nearest even, clamped to +-65504; hi + lo is within about 2^-22 of the mean).
 __global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__restrict__ k,
-                                                        __nv_bfloat16 *__restrict__ kbar_hi,
-                                                        __nv_bfloat16 *__restrict__ kbar_lo,
+                                                        __half *__restrict__ kbar_hi,
+                                                        __half *__restrict__ kbar_lo,
                                                         int64_t BH, int N, int nkb, int d) {
     const int ch = d >> 3;
     const int64_t total = BH * (int64_t)nkb * ch;
@@ -48,11 +49,11 @@ __global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__r
         for (int e = 0; e < 4; ++e) {
             float m0 = nt == 4 ? acc[2 * e] * 0.25f : __fdiv_rn(acc[2 * e], (float)nt);
             float m1 = nt == 4 ? acc[2 * e + 1] * 0.25f : __fdiv_rn(acc[2 * e + 1], (float)nt);
-            __nv_bfloat16 h0 = __float2bfloat16_rn(m0), h1 = __float2bfloat16_rn(m1);
-            __nv_bfloat16 l0 = __float2bfloat16_rn(m0 - __bfloat162float(h0));
-            __nv_bfloat16 l1 = __float2bfloat16_rn(m1 - __bfloat162float(h1));
-            hp[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lp[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+            const __half h0 = f16_sat(m0), h1 = f16_sat(m1);
+            const __half l0 = f16_sat(m0 - __half2float(h0));
+            const __half l1 = f16_sat(m1 - __half2float(h1));
+            hp[e] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+            lp[e] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
         }
         *reinterpret_cast<uint4 *>(kbar_hi + row * d + c * 8) = hi_u;
         *reinterpret_cast<uint4 *>(kbar_lo + row * d + c * 8) = lo_u;
@@ -97,7 +98,7 @@ struct KmeansSmem {
 template <int D>
 __global__ void __launch_bounds__(128, 4) absa_kmeans_kernel(
     const __nv_bfloat16 *__restrict__ q, int N, int nqb, int iters, float *__restrict__ mu_out,
-    __nv_bfloat16 *__restrict__ mu_hi, __nv_bfloat16 *__restrict__ mu_lo, float *__restrict__ w_out,
+    __half *__restrict__ mu_hi, __half *__restrict__ mu_lo, float *__restrict__ w_out,
     uint8_t *__restrict__ assign_out) {
     using S = KmeansSmem<D>;
     constexpr int NC = 8;
@@ -249,9 +250,9 @@ __global__ void __launch_bounds__(128, 4) absa_kmeans_kernel(
         const float v = mut[e * NC + c];
         const int64_t o = (row * NC + c) * D + e;
         mu_out[o] = v;
-        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        const __half h = f16_sat(v);
         mu_hi[o] = h;
-        mu_lo[o] = __float2bfloat16_rn(v - __bfloat162float(h));
+        mu_lo[o] = f16_sat(v - __half2float(h));
     }
     // final assignment: member lists of the last round
     for (int c = 0; c < NC; ++c)
@@ -263,9 +264,12 @@ __global__ void __launch_bounds__(128, 4) absa_kmeans_kernel(
 
 // One CTA per (b, h, group of 16 query blocks); the group's 128 centroid rows
 // (16 blocks x 8 clusters) stay in shared memory while tiles of 128 key blocks
-// stream through a 2-stage TMA ring.  Logits are mu . kbar computed as
-// hi*hi + hi*lo + lo*hi with three bf16 tcgen05 MMAs per k-step (error about
-// 2^-16 relative, far below the score tolerance).
+// stream through a 2-stage TMA ring.  Logits are mu_hi . (kbar_hi + kbar_lo)
+// with two fp16 tcgen05 MMAs per k-step: kbar is carried to about 2^-22 and
+// mu to fp16 (relative rounding 2^-12 on average), so a logit of the
+// workloads (|l| up to about 6 after scaling) is off by about 1e-4 at most,
+// an order below the 1e-3 score tolerance; both passes use the same product,
+// so pass 2 normalises exactly the logits pass 1 summed.
 //   pass 1: D[(qb,c), j] = mu . kbar   (A = centroids, B = key tile); the
 //           thread owning TMEM lane (qb,c) keeps an online max and sum of
 //           exp2 over j and ends with L = lse2 - log2(w) for its centroid;
@@ -280,7 +284,7 @@ template <int D>
 struct ScoreSmem {
     static constexpr int kRegions = D / 64;                 // 64-element SW128 regions
     static constexpr int kTile = 128 * 128;                 // one region of 128 rows (bytes)
-    static constexpr int kMuBytes = 2 * kRegions * kTile;   // hi + lo
+    static constexpr int kMuBytes = kRegions * kTile;       // hi only
     static constexpr int kKbBytes = 2 * kRegions * kTile;   // one stage, hi + lo
     static constexpr int kMuOff = 0;
     static constexpr int kKbOff = kMuBytes;
@@ -294,7 +298,7 @@ struct ScoreSmem {
 template <int D>
 __global__ void __launch_bounds__(320, 1) absa_score_kernel(
     const __grid_constant__ CUtensorMap tm_kb_hi, const __grid_constant__ CUtensorMap tm_kb_lo,
-    const __grid_constant__ CUtensorMap tm_mu_hi, const __grid_constant__ CUtensorMap tm_mu_lo,
+    const __grid_constant__ CUtensorMap tm_mu_hi,
     const float *__restrict__ w, float *__restrict__ scores, int nqb, int nkb, int groups,
     float scale_log2, int32_t *status) {
     using S = ScoreSmem<D>;
@@ -342,11 +346,8 @@ __global__ void __launch_bounds__(320, 1) absa_score_kernel(
             tma_prefetch_desc(&tm_kb_lo);
             mbar_arrive_expect_tx(mu_full, S::kMuBytes);
             const uint32_t mu_base = smem_u32(sm + S::kMuOff);
-            for (int r = 0; r < S::kRegions; ++r) {
+            for (int r = 0; r < S::kRegions; ++r)
                 tma_load_2d(mu_base + r * S::kTile, &tm_mu_hi, 64 * r, (int)mu_row0, mu_full);
-                tma_load_2d(mu_base + (S::kRegions + r) * S::kTile, &tm_mu_lo, 64 * r,
-                            (int)mu_row0, mu_full);
-            }
             for (int g = 0; g < 2 * T; ++g) {
                 const int st = g & 1;
                 const int t = g % T;
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(320, 1) absa_score_kernel(
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0);
+            constexpr uint32_t idesc = idesc_f16_f32(128, 128, 0);
             const uint32_t mu_base = smem_u32(sm + S::kMuOff);
             bool ok = mbar_wait(mu_full, 0, status, abort_flag);
             for (int g = 0; ok && g < 2 * T; ++g) {
@@ -379,17 +380,18 @@ __global__ void __launch_bounds__(320, 1) absa_score_kernel(
                 const uint32_t a_base = pass2 ? kb_base : mu_base;
                 const uint32_t b_base = pass2 ? mu_base : kb_base;
                 const uint32_t dt = tmem + buf * 128;
+                // pass 1: mu_hi . kbar_hi + mu_hi . kbar_lo (A = mu, B = key tile);
+                // pass 2: kbar_hi . mu_hi + kbar_lo . mu_hi (A = key tile, B = mu)
+                const uint32_t lo = S::kRegions * S::kTile;  // offset of the key tile's lo part
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
-                    const uint32_t lo = S::kRegions * S::kTile;
                     const uint64_t ah = sw128_desc(a_base + off, 16, 1024);
-                    const uint64_t al = sw128_desc(a_base + lo + off, 16, 1024);
                     const uint64_t bhd = sw128_desc(b_base + off, 16, 1024);
-                    const uint64_t bl = sw128_desc(b_base + lo + off, 16, 1024);
+                    const uint64_t a2 = pass2 ? sw128_desc(a_base + lo + off, 16, 1024) : ah;
+                    const uint64_t b2 = pass2 ? bhd : sw128_desc(b_base + lo + off, 16, 1024);
                     tc_mma_f16(dt, ah, bhd, idesc, ks > 0);
-                    tc_mma_f16(dt, ah, bl, idesc, 1);
-                    tc_mma_f16(dt, al, bhd, idesc, 1);
+                    tc_mma_f16(dt, a2, b2, idesc, 1);
                 }
                 tc_commit(d_full + buf);
                 tc_commit(kb_empty + st);
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(320, 1) absa_score_kernel(
 
 // ------------------------------------------------------------------ launchers
 
-cudaError_t launch_pool(const __nv_bfloat16 *k, __nv_bfloat16 *kbar_hi, __nv_bfloat16 *kbar_lo,
+cudaError_t launch_pool(const __nv_bfloat16 *k, __half *kbar_hi, __half *kbar_lo,
                         int64_t BH, int N, int nkb, int d, cudaStream_t stream) {
     const int64_t total = BH * (int64_t)nkb * (d / 8);
     int64_t blocks = (total + 255) / 256;
@@ -513,7 +515,7 @@ cudaError_t launch_pool(const __nv_bfloat16 *k, __nv_bfloat16 *kbar_hi, __nv_bfl
 
 template <int D>
 static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int iters,
-                                   float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
+                                   float *mu, __half *mu_hi, __half *mu_lo, float *w,
                                    uint8_t *assign, cudaStream_t stream) {
     const int smem = KmeansSmem<D>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(absa_kmeans_kernel<D>,
@@ -525,16 +527,16 @@ static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, int64_t BH, int N, in
 }
 
 cudaError_t launch_kmeans(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int d, int iters,
-                          float *mu, __nv_bfloat16 *mu_hi, __nv_bfloat16 *mu_lo, float *w,
+                          float *mu, __half *mu_hi, __half *mu_lo, float *w,
                           uint8_t *assign, cudaStream_t stream) {
     return d == 64 ? launch_kmeans_d<64>(q, BH, N, nqb, iters, mu, mu_hi, mu_lo, w, assign, stream)
                    : launch_kmeans_d<128>(q, BH, N, nqb, iters, mu, mu_hi, mu_lo, w, assign, stream);
 }
 
 template <int D>
-static cudaError_t launch_score_d(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c,
-                                  const CUtensorMap &dd, const float *w, float *scores, int64_t BH,
-                                  int nqb, int nkb, float scale_log2, int32_t *status,
+static cudaError_t launch_score_d(const CUtensorMap &kb_hi, const CUtensorMap &kb_lo,
+                                  const CUtensorMap &mu_hi, const float *w, float *scores,
+                                  int64_t BH, int nqb, int nkb, float scale_log2, int32_t *status,
                                   cudaStream_t stream) {
     const int smem = ScoreSmem<D>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(absa_score_kernel<D>,
@@ -542,19 +544,19 @@ static cudaError_t launch_score_d(const CUtensorMap &a, const CUtensorMap &b, co
     if (e != cudaSuccess) return e;
     const int groups = (nqb + 15) / 16;
     absa_score_kernel<D><<<(unsigned)(BH * groups), 320, smem, stream>>>(
-        a, b, c, dd, w, scores, nqb, nkb, groups, scale_log2, status);
+        kb_hi, kb_lo, mu_hi, w, scores, nqb, nkb, groups, scale_log2, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,
-                         const CUtensorMap &tm_mu_hi, const CUtensorMap &tm_mu_lo, const float *w,
-                         float *scores, int64_t BH, int nqb, int nkb, int d, float softmax_scale,
-                         int32_t *status, cudaStream_t stream) {
+                         const CUtensorMap &tm_mu_hi, const float *w, float *scores, int64_t BH,
+                         int nqb, int nkb, int d, float softmax_scale, int32_t *status,
+                         cudaStream_t stream) {
     const float scale_log2 = softmax_scale * 1.4426950408889634f;
-    return d == 64 ? launch_score_d<64>(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, scores, BH,
-                                        nqb, nkb, scale_log2, status, stream)
-                   : launch_score_d<128>(tm_kb_hi, tm_kb_lo, tm_mu_hi, tm_mu_lo, w, scores, BH,
-                                         nqb, nkb, scale_log2, status, stream);
+    return d == 64 ? launch_score_d<64>(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, scores, BH, nqb, nkb,
+                                        scale_log2, status, stream)
+                   : launch_score_d<128>(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, scores, BH, nqb, nkb,
+                                         scale_log2, status, stream);
 }
 
 }  // namespace absa

@@ -102,11 +102,11 @@ int32_t absa_plan_capacity(const absa_params *p);
 
 /* Bytes of workspace absa_select_scores / absa_select_plan need.  Layout,
  * each region starting at a 256-byte boundary in this order:
- *   kbar_hi  bf16 [B,H,NKB,d]   mean key of every 4-token block, high part
- *   kbar_lo  bf16 [B,H,NKB,d]   low part (kbar ~= hi + lo to 2^-17)
+ *   kbar_hi  fp16 [B,H,NKB,d]   mean key of every 4-token block, high part
+ *   kbar_lo  fp16 [B,H,NKB,d]   low part (kbar ~= hi + lo to about 2^-22)
  *   mu       f32  [B,H,NQB,8,d] final k-means centroids
- *   mu_hi    bf16 [B,H,NQB,8,d] split of mu for the tensor-core score
- *   mu_lo    bf16 [B,H,NQB,8,d]
+ *   mu_hi    fp16 [B,H,NQB,8,d] fp16(mu), the centroid operand of the score
+ *   mu_lo    fp16 [B,H,NQB,8,d] fp16(mu - mu_hi) (audit only)
  *   w        f32  [B,H,NQB,8]   centroid weights |c| / n_valid
  *   assign   u8   [B,H,NQB,128] final assignment (255 for padded rows)
  * The regions after kbar_lo are readable audit outputs of the last call.
@@ -120,7 +120,10 @@ size_t absa_workspace_bytes(const absa_params *p);
  * keep their centroid), weight each centroid by its share of the block's m
  * valid queries, and write
  *   scores[b,h,qb,j] = sum_c w_c * softmax_j(softmax_scale * mu_c . kbar_j)
- * (f32 [B,H,NQB,NKB], each row sums to 1).  ws must hold
+ * (f32 [B,H,NQB,NKB], each row sums to 1).  The products mu_c . kbar_j run
+ * on the tensor cores as fp16(mu_c) . (kbar_hi + kbar_lo); inputs whose
+ * magnitude exceeds the fp16 range (65504) are clamped to it, which only
+ * the accuracy of the scores can notice.  ws must hold
  * absa_workspace_bytes(p) bytes (ABSA_ERR_WORKSPACE otherwise). */
 absa_status absa_select_scores(const absa_params *p, const void *q, const void *k,
                                float *scores, void *ws, size_t ws_bytes, void *stream);

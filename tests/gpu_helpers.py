@@ -46,14 +46,16 @@ def ws_views(w, ws):
         out[name] = ws[off:off + n]
         off = (off + n + 255) // 256 * 256
     res = {
-        "kbar_hi": out["kbar_hi"].view(torch.bfloat16).reshape(w.B, w.H, w.nkb, d),
-        "kbar_lo": out["kbar_lo"].view(torch.bfloat16).reshape(w.B, w.H, w.nkb, d),
+        "kbar_hi": out["kbar_hi"].view(torch.float16).reshape(w.B, w.H, w.nkb, d),
+        "kbar_lo": out["kbar_lo"].view(torch.float16).reshape(w.B, w.H, w.nkb, d),
         "mu": out["mu"].view(torch.float32).reshape(w.B, w.H, w.nqb, 8, d),
+        "mu_hi": out["mu_hi"].view(torch.float16).reshape(w.B, w.H, w.nqb, 8, d),
+        "mu_lo": out["mu_lo"].view(torch.float16).reshape(w.B, w.H, w.nqb, 8, d),
         "w": out["w"].view(torch.float32).reshape(w.B, w.H, w.nqb, 8),
         "assign": out["assign"].reshape(w.B, w.H, w.nqb, 128),
     }
-    return {k: v.cpu().numpy() if k != "kbar_hi" and k != "kbar_lo" else v.float().cpu().numpy()
-            for k, v in res.items()}
+    halves = ("kbar_hi", "kbar_lo", "mu_hi", "mu_lo")
+    return {k: v.float().cpu().numpy() if k in halves else v.cpu().numpy() for k, v in res.items()}
 
 
 def plan_from_oracle(p, ref, device="cuda"):
