@@ -9,15 +9,13 @@ namespace absa {
 
 constexpr int kSampleMaxKvBlocks = 49152;
 
-// K1: mean key of every 4-token block as fp16 hi + lo.
-cudaError_t launch_pool(const __nv_bfloat16 *k, __half *kbar_hi, __half *kbar_lo,
-                        int64_t BH, int N, int nkb, int d, cudaStream_t stream);
-
-// K2: per-query-block k-means (8 clusters), centroids, their fp16 split,
-// weights and final assignment.
-cudaError_t launch_kmeans(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int d, int iters,
-                          float *mu, __half *mu_hi, __half *mu_lo, float *w,
-                          uint8_t *assign, cudaStream_t stream);
+// K1 + K2: per-query-block k-means (8 clusters): centroids, their fp16 split,
+// weights and final assignment; the same CTA also writes the mean key of the
+// 32 key blocks of its 128-token range as fp16 hi + lo.
+cudaError_t launch_kmeans_pool(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int64_t BH, int N,
+                               int nqb, int nkb, int d, int iters, float *mu, __half *mu_hi,
+                               __half *mu_lo, float *w, uint8_t *assign, __half *kbar_hi,
+                               __half *kbar_lo, cudaStream_t stream);
 
 // K3: block scores from the centroids (fp16 hi) and the key-block split (fp16 hi + lo).
 cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,

@@ -211,10 +211,9 @@ absa_status select_scores_run(const absa_params *p, const void *q, const void *k
         !make_map_f16(&tm_mu_hi, mu_hi, hr.nbh * dm.nqb * 8, p->d))
         return ABSA_ERR_CUDA;
 
-    cudaError_t e = launch_pool(kh, kb_hi, kb_lo, hr.nbh, p->N, dm.nkb, p->d, s);
-    if (e != cudaSuccess) return from_cuda(e);
-    e = launch_kmeans(qh, hr.nbh, p->N, dm.nqb, p->d, p->kmeans_iters, mu, mu_hi, mu_lo, w, assign,
-                      s);
+    cudaError_t e = launch_kmeans_pool(qh, kh, hr.nbh, p->N, dm.nqb, dm.nkb, p->d,
+                                       p->kmeans_iters, mu, mu_hi, mu_lo, w, assign, kb_hi, kb_lo,
+                                       s);
     if (e != cudaSuccess) return from_cuda(e);
     e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, sh, hr.nbh, dm.nqb, dm.nkb, p->d,
                      p->softmax_scale, status, s);

@@ -1,62 +1,48 @@
 // select.cu -- IBCS block selector on sm_100a (AB-Attention summary page,
 // "AB-Attention's three techniques", IBCS paragraph):
-//   K1 absa_pool_kernel    mean key of every 4-token block, split hi+lo bf16
-//   K2 absa_kmeans_kernel  per-128-query-block Lloyd k-means in shared memory
+//   K1 (in K2)             mean key of every 4-token block, split hi+lo fp16
+//   K2 absa_kmeans_kernel  per-128-query-block Lloyd k-means in shared memory,
+//                          plus the key-block means of the same token range
 //   K3 absa_score_kernel   weighted centroid softmax over all key blocks, on
-//                          tcgen05 tensor cores (3-product bf16 split, TMEM)
+//                          tcgen05 tensor cores (2-product fp16 split, TMEM)
 #include "absa_kernels.cuh"
 
 namespace absa {
 
 // ------------------------------------------------------------------------ K1
 
-// One thread per (row = (b,h,j), 8-element chunk): reads the 4 token rows of
-// block j (16-byte loads, a warp covers whole rows), averages in fp32 and
-// stores mean = hi + lo with hi = fp16(mean), lo = fp16(mean - hi) (round to
-// nearest even, clamped to +-65504; hi + lo is within about 2^-22 of the mean).
-__global__ void __launch_bounds__(256) absa_pool_kernel(const __nv_bfloat16 *__restrict__ k,
-                                                        __half *__restrict__ kbar_hi,
-                                                        __half *__restrict__ kbar_lo,
-                                                        int64_t BH, int N, int nkb, int d) {
-    const int ch = d >> 3;
-    const int64_t total = BH * (int64_t)nkb * ch;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int c = (int)(i % ch);
-        const int64_t row = i / ch;
-        const int64_t bh = row / nkb;
-        const int j = (int)(row % nkb);
-        const int t0 = 4 * j;
-        const int nt = min(4, N - t0);
-        const __nv_bfloat16 *src = k + ((bh * N + t0) * (int64_t)d) + c * 8;
-        float acc[8];
+// Mean of nt (1..4) token rows of one 8-element chunk (tokens summed in
+// ascending order in fp32, then times 1/4 or divided by nt) stored as
+// mean = hi + lo with hi = fp16(mean), lo = fp16(mean - hi) (round to nearest
+// even, clamped to +-65504; hi + lo is within about 2^-22 of the mean).  The
+// k-means kernel runs this for the 32 key blocks of its own 128-token range.
+__device__ __forceinline__ void pool_chunk(const uint4 (&u)[4], int nt, uint4 &hi_u, uint4 &lo_u) {
+    float acc[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        for (int t = 0; t < nt; ++t) {
-            uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)t * d));
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        if (t < nt) {
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u[t]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                float2 f = __bfloat1622float2(h2[e]);
+                const float2 f = __bfloat1622float2(h2[e]);
                 acc[2 * e] += f.x;
                 acc[2 * e + 1] += f.y;
             }
         }
-        uint4 hi_u, lo_u;
-        uint32_t *hp = reinterpret_cast<uint32_t *>(&hi_u);
-        uint32_t *lp = reinterpret_cast<uint32_t *>(&lo_u);
+    }
+    uint32_t *hp = reinterpret_cast<uint32_t *>(&hi_u);
+    uint32_t *lp = reinterpret_cast<uint32_t *>(&lo_u);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float m0 = nt == 4 ? acc[2 * e] * 0.25f : __fdiv_rn(acc[2 * e], (float)nt);
-            float m1 = nt == 4 ? acc[2 * e + 1] * 0.25f : __fdiv_rn(acc[2 * e + 1], (float)nt);
-            const __half h0 = f16_sat(m0), h1 = f16_sat(m1);
-            const __half l0 = f16_sat(m0 - __half2float(h0));
-            const __half l1 = f16_sat(m1 - __half2float(h1));
-            hp[e] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-            lp[e] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
-        }
-        *reinterpret_cast<uint4 *>(kbar_hi + row * d + c * 8) = hi_u;
-        *reinterpret_cast<uint4 *>(kbar_lo + row * d + c * 8) = lo_u;
+    for (int e = 0; e < 4; ++e) {
+        const float m0 = nt == 4 ? acc[2 * e] * 0.25f : __fdiv_rn(acc[2 * e], (float)nt);
+        const float m1 = nt == 4 ? acc[2 * e + 1] * 0.25f : __fdiv_rn(acc[2 * e + 1], (float)nt);
+        const __half h0 = f16_sat(m0), h1 = f16_sat(m1);
+        const __half l0 = f16_sat(m0 - __half2float(h0));
+        const __half l1 = f16_sat(m1 - __half2float(h1));
+        hp[e] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+        lp[e] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
     }
 }
 
@@ -96,10 +82,11 @@ struct KmeansSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(128, 4) absa_kmeans_kernel(
-    const __nv_bfloat16 *__restrict__ q, int N, int nqb, int iters, float *__restrict__ mu_out,
-    __half *__restrict__ mu_hi, __half *__restrict__ mu_lo, float *__restrict__ w_out,
-    uint8_t *__restrict__ assign_out) {
+__global__ void __launch_bounds__(128, 5) absa_kmeans_kernel(
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k, int N, int nqb,
+    int nkb, int iters, float *__restrict__ mu_out, __half *__restrict__ mu_hi,
+    __half *__restrict__ mu_lo, float *__restrict__ w_out, uint8_t *__restrict__ assign_out,
+    __half *__restrict__ kbar_hi, __half *__restrict__ kbar_lo) {
     using S = KmeansSmem<D>;
     constexpr int NC = 8;
     extern __shared__ __align__(16) uint8_t kms[];
@@ -131,6 +118,39 @@ __global__ void __launch_bounds__(128, 4) absa_kmeans_kernel(
         for (int u = 0; u < CPR; ++u) {
             const int idx = tid + 128 * u, r = idx / CPR, c = idx % CPR;
             if (r < m) *reinterpret_cast<uint4 *>(xs + r * XR + c * 8) = v[u];
+        }
+    }
+    {
+        // K1: pooled keys of the same 128-token range, key blocks 32 qb .. 32 qb + 31,
+        // two chunks per thread at a time with all their loads issued first
+        constexpr int UPT = CPR / 4;  // 32 blocks x CPR chunks over 128 threads
+        constexpr int BATCH = UPT < 2 ? UPT : 2;
+        const int jb0 = qb * 32;
+        const int nblk = min(32, nkb - jb0);
+        const __nv_bfloat16 *ksrc = k + (bh * N + (int64_t)qb * 128) * D;
+#pragma unroll
+        for (int i0 = 0; i0 < UPT; i0 += BATCH) {
+            uint4 kv[BATCH][4];
+            int nt[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                const int u = tid + 128 * (i0 + i), blk = u / CPR, c = u % CPR;
+                nt[i] = blk < nblk ? min(4, N - 4 * (jb0 + blk)) : 0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    if (t < nt[i])
+                        kv[i][t] = __ldg(reinterpret_cast<const uint4 *>(ksrc + (int64_t)(4 * blk + t) * D) + c);
+            }
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                if (nt[i] == 0) continue;
+                const int u = tid + 128 * (i0 + i), blk = u / CPR, c = u % CPR;
+                uint4 hi_u, lo_u;
+                pool_chunk(kv[i], nt[i], hi_u, lo_u);
+                const int64_t o = (bh * nkb + jb0 + blk) * (int64_t)D + c * 8;
+                *reinterpret_cast<uint4 *>(kbar_hi + o) = hi_u;
+                *reinterpret_cast<uint4 *>(kbar_lo + o) = lo_u;
+            }
         }
     }
     __syncthreads();
@@ -503,34 +523,28 @@ __global__ void __launch_bounds__(320, 1) absa_score_kernel(
 
 // ------------------------------------------------------------------ launchers
 
-cudaError_t launch_pool(const __nv_bfloat16 *k, __half *kbar_hi, __half *kbar_lo,
-                        int64_t BH, int N, int nkb, int d, cudaStream_t stream) {
-    const int64_t total = BH * (int64_t)nkb * (d / 8);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    if (blocks < 1) blocks = 1;
-    absa_pool_kernel<<<(unsigned)blocks, 256, 0, stream>>>(k, kbar_hi, kbar_lo, BH, N, nkb, d);
-    return cudaGetLastError();
-}
-
 template <int D>
-static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int iters,
-                                   float *mu, __half *mu_hi, __half *mu_lo, float *w,
-                                   uint8_t *assign, cudaStream_t stream) {
+static cudaError_t launch_kmeans_d(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int64_t BH,
+                                   int N, int nqb, int nkb, int iters, float *mu, __half *mu_hi,
+                                   __half *mu_lo, float *w, uint8_t *assign, __half *kbar_hi,
+                                   __half *kbar_lo, cudaStream_t stream) {
     const int smem = KmeansSmem<D>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(absa_kmeans_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    absa_kmeans_kernel<D><<<(unsigned)(BH * nqb), 128, smem, stream>>>(q, N, nqb, iters, mu, mu_hi,
-                                                                      mu_lo, w, assign);
+    absa_kmeans_kernel<D><<<(unsigned)(BH * nqb), 128, smem, stream>>>(
+        q, k, N, nqb, nkb, iters, mu, mu_hi, mu_lo, w, assign, kbar_hi, kbar_lo);
     return cudaGetLastError();
 }
 
-cudaError_t launch_kmeans(const __nv_bfloat16 *q, int64_t BH, int N, int nqb, int d, int iters,
-                          float *mu, __half *mu_hi, __half *mu_lo, float *w,
-                          uint8_t *assign, cudaStream_t stream) {
-    return d == 64 ? launch_kmeans_d<64>(q, BH, N, nqb, iters, mu, mu_hi, mu_lo, w, assign, stream)
-                   : launch_kmeans_d<128>(q, BH, N, nqb, iters, mu, mu_hi, mu_lo, w, assign, stream);
+cudaError_t launch_kmeans_pool(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int64_t BH, int N,
+                               int nqb, int nkb, int d, int iters, float *mu, __half *mu_hi,
+                               __half *mu_lo, float *w, uint8_t *assign, __half *kbar_hi,
+                               __half *kbar_lo, cudaStream_t stream) {
+    return d == 64 ? launch_kmeans_d<64>(q, k, BH, N, nqb, nkb, iters, mu, mu_hi, mu_lo, w, assign,
+                                         kbar_hi, kbar_lo, stream)
+                   : launch_kmeans_d<128>(q, k, BH, N, nqb, nkb, iters, mu, mu_hi, mu_lo, w,
+                                          assign, kbar_hi, kbar_lo, stream);
 }
 
 template <int D>

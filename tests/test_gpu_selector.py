@@ -1,4 +1,4 @@
-"""GPU IBCS selector (K1 pool, K2 k-means, K3 score) against the oracle.
+"""GPU IBCS selector (key pooling and k-means in K2, K3 score) against the oracle.
 
 Criteria: k-means centroids, weights and assignments bit-equal (both sides
 take the decisions in fp32 with the same arithmetic order); pooled keys as an
