@@ -15,11 +15,19 @@
 
 namespace absa {
 
-__device__ __forceinline__ uint64_t quantise_score(float s) {
+// q - 1 as a u32 (q = max(1, floor(s 2^32)) <= 2^32).
+__device__ __forceinline__ uint32_t quantise_m1(float s) {
     const float x = s * 4294967296.0f;  // exact power-of-two scaling
-    if (!(x >= 1.0f)) return 1ull;      // NaN, negative, or below one unit
-    if (x >= 4294967296.0f) return 1ull << 32;
-    return (uint64_t)x;                 // floor for x >= 1
+    if (!(x >= 1.0f)) return 0u;        // NaN, negative, or below one unit
+    if (x >= 4294967296.0f) return 0xFFFFFFFFu;
+    return __float2uint_rz(x) - 1u;     // floor for 1 <= x < 2^32
+}
+
+// Threshold t - 1 of "q >= t" on q - 1 as a u32, or `never` when t - 1 exceeds
+// every q - 1 (q <= 2^32).
+__device__ __forceinline__ uint32_t q_threshold_m1(uint64_t t, bool &never) {
+    never = t - 1 > 0xFFFFFFFFull;
+    return never ? 0xFFFFFFFFu : (uint32_t)(t - 1);
 }
 
 constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;  // SplitMix64 increment
@@ -155,9 +163,9 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
         for (int u = 0; u < 8; ++u) {
             const int j = (g + u) * 32 + lane;
             if (g + u < g1 && j < nkb) {
-                const uint64_t qj = quantise_score(sv[u]);
-                qm1[j] = (uint32_t)(qj - 1);
-                R += qj;
+                const uint32_t qm = quantise_m1(sv[u]);
+                qm1[j] = qm;
+                R += (uint64_t)qm + 1;
             }
         }
     }
@@ -165,20 +173,25 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     const uint64_t R0 = R;
     const uint64_t nn = (uint64_t)n;
 
-    // round 1 over every block (r = n), listing the candidates for later rounds
+    // round 1 over every block (r = n), listing the candidates for later rounds:
+    // n q >= R0 <=> q >= ceil(R0 / n), and 2 n q >= R0 <=> q >= ceil(R0 / (2 n)),
+    // compared on q - 1 in 32 bits
     const uint32_t below = (1u << lane) - 1u;
+    bool never_cap, never_cand;
+    const uint32_t t_cap = q_threshold_m1((R0 + nn - 1) / nn, never_cap);
+    const uint32_t t_cand = q_threshold_m1((R0 + 2 * nn - 1) / (2 * nn), never_cand);
     uint64_t capsum = 0;
     int capcnt = 0;
     for (int g = g0; g < g1; ++g) {
         const int j = g * 32 + lane;
         bool newcap = false, is_cand = false;
         if (j < nkb) {
-            const uint64_t q = (uint64_t)qm1[j] + 1;
-            if (nn * q >= R0) {
+            const uint32_t qm = qm1[j];
+            if (!never_cap && qm >= t_cap) {
                 newcap = true;
-                capsum += q;
+                capsum += (uint64_t)qm + 1;
                 ++capcnt;
-            } else if (2 * nn * q >= R0) {
+            } else if (!never_cand && qm >= t_cand) {
                 is_cand = true;
             }
         }
