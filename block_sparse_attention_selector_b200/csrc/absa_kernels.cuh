@@ -17,11 +17,15 @@ cudaError_t launch_kmeans_pool(const __nv_bfloat16 *q, const __nv_bfloat16 *k, i
                                __half *mu_lo, float *w, uint8_t *assign, __half *kbar_hi,
                                __half *kbar_lo, cudaStream_t stream);
 
-// K3: block scores from the centroids (fp16 hi) and the key-block split (fp16 hi + lo).
+// K3: block scores from the centroids (fp16 hi) and the key-block split (fp16
+// hi + lo), in three launches (partial log-sum-exp per key range, combine,
+// scores).  part_m/part_s hold [BH, score_key_ranges(nkb), NQB*8] floats, L
+// [BH, NQB*8].
+int score_key_ranges(int nkb);
 cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,
-                         const CUtensorMap &tm_mu_hi, const float *w, float *scores, int64_t BH,
-                         int nqb, int nkb, int d, float softmax_scale, int32_t *status,
-                         cudaStream_t stream);
+                         const CUtensorMap &tm_mu_hi, const float *w, float *part_m,
+                         float *part_s, float *L, float *scores, int64_t BH, int nqb, int nkb,
+                         int d, float softmax_scale, int32_t *status, cudaStream_t stream);
 
 // K4: SIP plan rows from a score array.
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,

@@ -29,7 +29,7 @@ Dims dims_of(const absa_params *p) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-    size_t kbar_hi, kbar_lo, mu, mu_hi, mu_lo, w, assign, total;
+    size_t kbar_hi, kbar_lo, mu, mu_hi, mu_lo, w, assign, part_m, part_s, lse, total;
 };
 
 WsLayout ws_layout(const absa_params *p) {
@@ -49,6 +49,10 @@ WsLayout ws_layout(const absa_params *p) {
     L.mu_lo = take((size_t)dm.BH * dm.nqb * 8 * d * 2);
     L.w = take((size_t)dm.BH * dm.nqb * 8 * 4);
     L.assign = take((size_t)dm.BH * dm.nqb * 128);
+    const size_t parts = (size_t)dm.BH * score_key_ranges(dm.nkb) * dm.nqb * 8 * 4;
+    L.part_m = take(parts);
+    L.part_s = take(parts);
+    L.lse = take((size_t)dm.BH * dm.nqb * 8 * 4);
     L.total = off;
     return L;
 }
@@ -201,6 +205,10 @@ absa_status select_scores_run(const absa_params *p, const void *q, const void *k
     auto *mu_lo = reinterpret_cast<__half *>(w8 + L.mu_lo) + hr.bh0 * dm.nqb * 8 * d;
     auto *w = reinterpret_cast<float *>(w8 + L.w) + hr.bh0 * dm.nqb * 8;
     auto *assign = w8 + L.assign + hr.bh0 * dm.nqb * 128;
+    const int64_t nkr = score_key_ranges(dm.nkb);
+    auto *part_m = reinterpret_cast<float *>(w8 + L.part_m) + hr.bh0 * nkr * dm.nqb * 8;
+    auto *part_s = reinterpret_cast<float *>(w8 + L.part_s) + hr.bh0 * nkr * dm.nqb * 8;
+    auto *lse = reinterpret_cast<float *>(w8 + L.lse) + hr.bh0 * dm.nqb * 8;
     const auto *qh = static_cast<const __nv_bfloat16 *>(q) + hr.bh0 * p->N * d;
     const auto *kh = static_cast<const __nv_bfloat16 *>(k) + hr.bh0 * p->N * d;
     float *sh = scores + hr.bh0 * dm.nqb * (int64_t)dm.nkb;
@@ -215,7 +223,8 @@ absa_status select_scores_run(const absa_params *p, const void *q, const void *k
                                        p->kmeans_iters, mu, mu_hi, mu_lo, w, assign, kb_hi, kb_lo,
                                        s);
     if (e != cudaSuccess) return from_cuda(e);
-    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, sh, hr.nbh, dm.nqb, dm.nkb, p->d,
+    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, part_m, part_s, lse, sh, hr.nbh, dm.nqb,
+                     dm.nkb, p->d,
                      p->softmax_scale, status, s);
     return from_cuda(e);
 }

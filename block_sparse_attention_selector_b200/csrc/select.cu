@@ -3,8 +3,7 @@
 //   K1 (in K2)             mean key of every 4-token block, split hi+lo fp16
 //   K2 absa_kmeans_kernel  per-128-query-block Lloyd k-means in shared memory,
 //                          plus the key-block means of the same token range
-//   K3 absa_score_kernel   weighted centroid softmax over all key blocks, on
-//                          tcgen05 tensor cores (2-product fp16 split, TMEM)
+// (the block score from these centroids is in score.cu)
 #include "absa_kernels.cuh"
 
 namespace absa {
@@ -280,247 +279,6 @@ __global__ void __launch_bounds__(128, 5) absa_kmeans_kernel(
     if (tid >= m) assign_out[row * 128 + tid] = (uint8_t)255;
 }
 
-// ------------------------------------------------------------------------ K3
-
-// One CTA per (b, h, group of 16 query blocks); the group's 128 centroid rows
-// (16 blocks x 8 clusters) stay in shared memory while tiles of 128 key blocks
-// stream through a 2-stage TMA ring.  Logits are mu_hi . (kbar_hi + kbar_lo)
-// with two fp16 tcgen05 MMAs per k-step: kbar is carried to about 2^-22 and
-// mu to fp16 (relative rounding 2^-12 on average), so a logit of the
-// workloads (|l| up to about 6 after scaling) is off by about 1e-4 at most,
-// an order below the 1e-3 score tolerance; both passes use the same product,
-// so pass 2 normalises exactly the logits pass 1 summed.
-//   pass 1: D[(qb,c), j] = mu . kbar   (A = centroids, B = key tile); the
-//           thread owning TMEM lane (qb,c) keeps an online max and sum of
-//           exp2 over j and ends with L = lse2 - log2(w) for its centroid;
-//   pass 2: D[j, (qb,c)] = kbar . mu   (A = key tile, B = centroids); the
-//           thread owning lane j forms s_j = sum_c exp2(scaled logit - L_c)
-//           for each of the 16 query blocks and stores it.
-// Warps: 0 TMA producer, 1 MMA issuer (+TMEM owner), 2..9 epilogue in two
-// warpgroups: warpgroup g takes columns 64g..64g+63 of every tile (pass 1:
-// its own online max/sum, merged with the other half once at the end; pass
-// 2: query blocks 8g..8g+7 of the group).
-template <int D>
-struct ScoreSmem {
-    static constexpr int kRegions = D / 64;                 // 64-element SW128 regions
-    static constexpr int kTile = 128 * 128;                 // one region of 128 rows (bytes)
-    static constexpr int kMuBytes = kRegions * kTile;       // hi only
-    static constexpr int kKbBytes = 2 * kRegions * kTile;   // one stage, hi + lo
-    static constexpr int kMuOff = 0;
-    static constexpr int kKbOff = kMuBytes;
-    static constexpr int kLOff = kKbOff + 2 * kKbBytes;     // f32 [128] L per centroid row
-    static constexpr int kXOff = kLOff + 128 * 4;           // f32 [2][2][128] pass-1 halves
-    static constexpr int kBarOff = kXOff + 4 * 128 * 4;
-    static constexpr int kBytes = kBarOff + 16 * 8 + 16;
-    static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
-};
-
-template <int D>
-__global__ void __launch_bounds__(320, 1) absa_score_kernel(
-    const __grid_constant__ CUtensorMap tm_kb_hi, const __grid_constant__ CUtensorMap tm_kb_lo,
-    const __grid_constant__ CUtensorMap tm_mu_hi,
-    const float *__restrict__ w, float *__restrict__ scores, int nqb, int nkb, int groups,
-    float scale_log2, int32_t *status) {
-    using S = ScoreSmem<D>;
-    extern __shared__ uint8_t score_smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(score_smem_raw) + 1023) & ~uintptr_t(1023));
-    float *Ltab = reinterpret_cast<float *>(sm + S::kLOff);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::kBarOff);
-    uint64_t *mu_full = bars + 0;
-    uint64_t *kb_full = bars + 1;   // [2]
-    uint64_t *kb_empty = bars + 3;  // [2]
-    uint64_t *d_full = bars + 5;    // [2]
-    uint64_t *d_empty = bars + 7;   // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 10);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t bh = blockIdx.x / groups;
-    const int qb0 = (blockIdx.x % groups) * 16;
-    const int T = (nkb + 127) / 128;
-    const int64_t kv_row0 = bh * nkb;
-    const int64_t mu_row0 = (bh * nqb + qb0) * 8;
-
-    if (threadIdx.x == 0) {
-        mbar_init(mu_full, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(kb_full + s, 1);
-            mbar_init(kb_empty + s, 1);
-            mbar_init(d_full + s, 1);
-            mbar_init(d_empty + s, 8);
-        }
-        *abort_flag = 0;
-        mbar_fence_init();
-    }
-    if (warp == 1) tmem_alloc(tmem_slot, 256);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_kb_hi);
-            tma_prefetch_desc(&tm_kb_lo);
-            mbar_arrive_expect_tx(mu_full, S::kMuBytes);
-            const uint32_t mu_base = smem_u32(sm + S::kMuOff);
-            for (int r = 0; r < S::kRegions; ++r)
-                tma_load_2d(mu_base + r * S::kTile, &tm_mu_hi, 64 * r, (int)mu_row0, mu_full);
-            for (int g = 0; g < 2 * T; ++g) {
-                const int st = g & 1;
-                const int t = g % T;
-                if (g >= 2 && !mbar_wait(kb_empty + st, ((g - 2) >> 1) & 1, status, abort_flag))
-                    break;
-                mbar_arrive_expect_tx(kb_full + st, S::kKbBytes);
-                const uint32_t kb_base = smem_u32(sm + S::kKbOff + st * S::kKbBytes);
-                const int y = (int)(kv_row0 + (int64_t)t * 128);
-                for (int r = 0; r < S::kRegions; ++r) {
-                    tma_load_2d(kb_base + r * S::kTile, &tm_kb_hi, 64 * r, y, kb_full + st);
-                    tma_load_2d(kb_base + (S::kRegions + r) * S::kTile, &tm_kb_lo, 64 * r, y,
-                                kb_full + st);
-                }
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16_f32(128, 128, 0);
-            const uint32_t mu_base = smem_u32(sm + S::kMuOff);
-            bool ok = mbar_wait(mu_full, 0, status, abort_flag);
-            for (int g = 0; ok && g < 2 * T; ++g) {
-                const int st = g & 1;
-                const int buf = g & 1;
-                const bool pass2 = g >= T;
-                if (!mbar_wait(kb_full + st, (g >> 1) & 1, status, abort_flag)) break;
-                if (g >= 2 && !mbar_wait(d_empty + buf, ((g - 2) >> 1) & 1, status, abort_flag))
-                    break;
-                tc_fence_after();
-                const uint32_t kb_base = smem_u32(sm + S::kKbOff + st * S::kKbBytes);
-                const uint32_t a_base = pass2 ? kb_base : mu_base;
-                const uint32_t b_base = pass2 ? mu_base : kb_base;
-                const uint32_t dt = tmem + buf * 128;
-                // pass 1: mu_hi . kbar_hi + mu_hi . kbar_lo (A = mu, B = key tile);
-                // pass 2: kbar_hi . mu_hi + kbar_lo . mu_hi (A = key tile, B = mu)
-                const uint32_t lo = S::kRegions * S::kTile;  // offset of the key tile's lo part
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
-                    const uint64_t ah = sw128_desc(a_base + off, 16, 1024);
-                    const uint64_t bhd = sw128_desc(b_base + off, 16, 1024);
-                    const uint64_t a2 = pass2 ? sw128_desc(a_base + lo + off, 16, 1024) : ah;
-                    const uint64_t b2 = pass2 ? bhd : sw128_desc(b_base + lo + off, 16, 1024);
-                    tc_mma_f16(dt, ah, bhd, idesc, ks > 0);
-                    tc_mma_f16(dt, a2, b2, idesc, 1);
-                }
-                tc_commit(d_full + buf);
-                tc_commit(kb_empty + st);
-            }
-        }
-    } else {
-        // epilogue: thread <-> TMEM lane; warp w owns lane quarter w % 4
-        const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;  // column half (warpgroup)
-        const int lrow = quarter * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + half * 64;
-        float *xch = reinterpret_cast<float *>(sm + S::kXOff);  // [max|sum][half][row]
-        bool ok = true;
-        // pass 1: online log-sum-exp over this half's key blocks of the row
-        float mx = -INFINITY, sum = 0.f;
-        for (int t = 0; t < T && ok; ++t) {
-            const int buf = t & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(d_full + buf, (t >> 1) & 1, status, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t v[2][32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(d_empty + buf);
-            const int ncols = min(64, nkb - t * 128 - half * 64);
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (ch * 32 + i < ncols) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(v[ch][i]));
-            const float tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            if (tmax > mx) {
-                sum *= ex2((mx - tmax) * scale_log2);
-                mx = tmax;
-            }
-            const float moff = -mx * scale_log2;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (ch * 32 + i < ncols)
-                        a4[i & 3] += ex2(__fmaf_rn(__uint_as_float(v[ch][i]), scale_log2, moff));
-            sum += (a4[0] + a4[1]) + (a4[2] + a4[3]);
-        }
-        // merge the two halves of each row (every epilogue thread passes here once)
-        xch[half * 128 + lrow] = mx;
-        xch[256 + half * 128 + lrow] = sum;
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        {
-            const float m0 = xch[lrow], m1 = xch[128 + lrow];
-            const float mm = fmaxf(m0, m1);
-            const float s0 = xch[256 + lrow], s1 = xch[384 + lrow];
-            const float tot = (m0 == -INFINITY ? 0.f : s0 * ex2((m0 - mm) * scale_log2)) +
-                              (m1 == -INFINITY ? 0.f : s1 * ex2((m1 - mm) * scale_log2));
-            const int qb = qb0 + (lrow >> 3);
-            const float wc = qb < nqb ? w[(bh * nqb + qb) * 8 + (lrow & 7)] : 0.f;
-            const float lse2 = mm * scale_log2 + log2f(tot);
-            if (half == 0) Ltab[lrow] = wc > 0.f ? lse2 - log2f(wc) : INFINITY;
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        // pass 2: combine the 8 centroids of each of this half's query blocks
-        for (int t = 0; t < T && ok; ++t) {
-            const int g = T + t;
-            const int buf = g & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(d_full + buf, (g >> 1) & 1, status, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t v[2][32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) tmem_ld32(lane_addr + buf * 128 + ch * 32, v[ch]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(d_empty + buf);
-            const int j = t * 128 + lrow;
-            if (j < nkb) {
-#pragma unroll
-                for (int qbl = 0; qbl < 8; ++qbl) {
-                    const int qb = qb0 + half * 8 + qbl;
-                    if (qb >= nqb) continue;
-                    const float4 L0 = *reinterpret_cast<const float4 *>(Ltab + (half * 8 + qbl) * 8);
-                    const float4 L1 = *reinterpret_cast<const float4 *>(Ltab + (half * 8 + qbl) * 8 + 4);
-                    const float Lc[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
-                    float s2[2] = {0.f, 0.f};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int col = qbl * 8 + c;
-                        s2[c & 1] += ex2(__fmaf_rn(__uint_as_float(v[col >> 5][col & 31]),
-                                                   scale_log2, -Lc[c]));
-                    }
-                    scores[(bh * nqb + qb) * (int64_t)nkb + j] = s2[0] + s2[1];
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, 256);
-    }
-}
-
 // ------------------------------------------------------------------ launchers
 
 template <int D>
@@ -545,32 +303,6 @@ cudaError_t launch_kmeans_pool(const __nv_bfloat16 *q, const __nv_bfloat16 *k, i
                                          kbar_hi, kbar_lo, stream)
                    : launch_kmeans_d<128>(q, k, BH, N, nqb, nkb, iters, mu, mu_hi, mu_lo, w,
                                           assign, kbar_hi, kbar_lo, stream);
-}
-
-template <int D>
-static cudaError_t launch_score_d(const CUtensorMap &kb_hi, const CUtensorMap &kb_lo,
-                                  const CUtensorMap &mu_hi, const float *w, float *scores,
-                                  int64_t BH, int nqb, int nkb, float scale_log2, int32_t *status,
-                                  cudaStream_t stream) {
-    const int smem = ScoreSmem<D>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(absa_score_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    const int groups = (nqb + 15) / 16;
-    absa_score_kernel<D><<<(unsigned)(BH * groups), 320, smem, stream>>>(
-        kb_hi, kb_lo, mu_hi, w, scores, nqb, nkb, groups, scale_log2, status);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_lo,
-                         const CUtensorMap &tm_mu_hi, const float *w, float *scores, int64_t BH,
-                         int nqb, int nkb, int d, float softmax_scale, int32_t *status,
-                         cudaStream_t stream) {
-    const float scale_log2 = softmax_scale * 1.4426950408889634f;
-    return d == 64 ? launch_score_d<64>(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, scores, BH, nqb, nkb,
-                                        scale_log2, status, stream)
-                   : launch_score_d<128>(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, scores, BH, nqb, nkb,
-                                         scale_log2, status, stream);
 }
 
 }  // namespace absa

@@ -109,6 +109,13 @@ int32_t absa_plan_capacity(const absa_params *p);
  *   mu_lo    fp16 [B,H,NQB,8,d] fp16(mu - mu_hi) (audit only)
  *   w        f32  [B,H,NQB,8]   centroid weights |c| / n_valid
  *   assign   u8   [B,H,NQB,128] final assignment (255 for padded rows)
+ *   part_m   f32  [B,H,NKR,NQB*8] per key range of 256 key blocks
+ *                               (NKR = ceil(NKB/256)) and centroid row: the
+ *                               largest logit mu . kbar over the range
+ *   part_s   f32  [B,H,NKR,NQB*8] sum over the range of exp of the scaled
+ *                               logit minus that largest one (base 2)
+ *   lse      f32  [B,H,NQB*8]   L = log2-sum-exp of the scaled logits over
+ *                               all key blocks minus log2(w) (+inf if w = 0)
  * The regions after kbar_lo are readable audit outputs of the last call.
  * Returns 0 if p is invalid. */
 size_t absa_workspace_bytes(const absa_params *p);
