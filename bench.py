@@ -393,7 +393,7 @@ def run_ours(args):
             "e2e": {"value": e2e_ms, "unit": "ms",
                     "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2,
                     "api": "absa_step_host", "heads_per_run": args.e2e_heads_per_run},
-            "gpu_launches": 4 * K,
+            "gpu_launches": 6 * K,
             "clocks": clk,
         }
     if world > 1:
