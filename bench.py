@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads (profiling captures); 0 = all 40")
     ap.add_argument("--dense-reps", type=int, default=3)
+    ap.add_argument("--workload", default="wan480", choices=WORKLOADS,
+                    help="layer to time: Wan2.1 480p (the default and the headline), Wan2.1 720p "
+                         "or HunyuanVideo 720p")
     ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic"],
                     help="SIP design: Poisson draws (default) or systematic (exactly n blocks)")
     ap.add_argument("--harness", action="store_true",
@@ -60,10 +63,14 @@ def parse():
     return ap.parse_args()
 
 
-def workload(heads=0):
+WORKLOADS = ("wan480", "wan720", "hunyuan720")
+
+
+def workload(heads=0, name="wan480"):
     from block_sparse_attention_selector_b200 import synthetic
 
-    w = synthetic.WAN480
+    w = {"wan480": synthetic.WAN480, "wan720": synthetic.WAN720,
+         "hunyuan720": synthetic.HUNYUAN720}[name]
     if heads:
         import dataclasses
 
@@ -123,7 +130,7 @@ def run_reference(args):
         return 0
     from block_sparse_attention_selector_b200 import synthetic
 
-    w = workload()
+    w = workload(name=args.workload)
     q, k, v = synthetic.layer_qkv_bits(w)
     import oracle
 
@@ -218,8 +225,9 @@ def measured_peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def recorded_traffic(kernel_src):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+def recorded_traffic(kernel_src, w):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source and
+    was taken on this layer (the 40-head Wan2.1 480p layer)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -228,7 +236,8 @@ def recorded_traffic(kernel_src):
     with open(kernel_src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()[:16]
     ent = rec.get("sparse_attention")
-    if ent and ent.get("source_sha256_16") == digest:
+    if ent and ent.get("source_sha256_16") == digest and ent.get("workload", w.name) == w.name \
+            and w.H == 40 and w.name.startswith("wan2.1_480p"):
         return ent.get("dram_bytes_per_launch")
     return None
 
@@ -249,7 +258,7 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    w = workload(args.heads)
+    w = workload(args.heads, args.workload)
     q_bits, k_bits, v_bits = synthetic.layer_qkv_bits(w)
 
     def to_dev(b):
@@ -388,7 +397,8 @@ def run_ours(args):
                                         f"{float(tot.sum()):.0f} ms)",
                          "frac_of_burst_peak": achieved_tf / burst_tf,
                          "traffic": recorded_traffic(os.path.join(
-                             ROOT, "block_sparse_attention_selector_b200", "csrc", "attention.cu")),
+                             ROOT, "block_sparse_attention_selector_b200", "csrc", "attention.cu"),
+                             w),
                          "algorithmic_flops_per_launch": attn_flops},
             "e2e": {"value": e2e_ms, "unit": "ms",
                     "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2,
@@ -423,7 +433,7 @@ def run_sweep(args):
     from block_sparse_attention_selector_b200 import synthetic
 
     dev = torch.device("cuda", 0)
-    w = workload(args.heads)
+    w = workload(args.heads, args.workload)
     q_bits, k_bits, v_bits = synthetic.layer_qkv_bits(w)
 
     def to_dev(b):

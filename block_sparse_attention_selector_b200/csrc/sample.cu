@@ -64,10 +64,8 @@ __device__ __forceinline__ uint64_t submod(uint64_t x, uint64_t y, uint64_t R) {
     return x >= y ? x - y : x + R - y;
 }
 
-constexpr int kSampleThreads = 256;
-constexpr int kSampleWarps = kSampleThreads / 32;
-
-// Block-wide sum of a u64 and an int; result broadcast to every thread.
+// Block-wide sum of a u64 and an int over WARPS warps; result broadcast to every thread.
+template <int WARPS>
 __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a, int *red_b) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -84,7 +82,7 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
     a = 0;
     b = 0;
 #pragma unroll
-    for (int w = 0; w < kSampleWarps; ++w) {
+    for (int w = 0; w < WARPS; ++w) {
         a += red_a[w];
         b += red_b[w];
     }
@@ -105,10 +103,13 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
 // the list, so warp 0 runs those rounds over the list alone.  If the list
 // overflows or the threshold falls below the half, the remaining rounds scan
 // every block.  Either way the rounds are exactly those of the definition.
-__global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
+template <int WARPS>
+__global__ void __launch_bounds__(32 * WARPS) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
     uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, bool systematic) {
+    constexpr int kSampleWarps = WARPS;
+    constexpr int kSampleThreads = 32 * WARPS;
     extern __shared__ __align__(16) uint32_t samp_smem[];
     const int ngroups = (nkb + 31) >> 5;
     const int ngp = (ngroups + 7) & ~7;             // groups rounded up to whole 256-block
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
             }
         }
     }
-    block_sum2(R, dummy, red_a, red_b);
+    block_sum2<WARPS>(R, dummy, red_a, red_b);
     const uint64_t R0 = R;
     const uint64_t nn = (uint64_t)n;
 
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
             if (is_cand && p < kCandMax) cand[p] = (uint32_t)j;
         }
     }
-    block_sum2(capsum, capcnt, red_a, red_b);
+    block_sum2<WARPS>(capsum, capcnt, red_a, red_b);
     int n_capped = capcnt;
     uint64_t r = nn - (uint64_t)n_capped;
     R = R0 - capsum;
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
                     grew += lane == 0 ? __popc(nb) : 0;
                 }
             }
-            block_sum2(newsum, grew, red_a, red_b);
+            block_sum2<WARPS>(newsum, grew, red_a, red_b);
             if (grew == 0) break;
             n_capped += grew;
             r = nn - (uint64_t)n_capped;
@@ -428,6 +429,19 @@ __global__ void __launch_bounds__(kSampleThreads) absa_sample_kernel(
     }
 }
 
+template <int WARPS>
+static cudaError_t launch_sample_w(const float *scores, int64_t rows, int nkb, int64_t n,
+                                   uint64_t seed, bool systematic, int cap, int32_t *counts,
+                                   int32_t *kv_index, float *log_pi, uint64_t *r_R,
+                                   int32_t *status, int64_t row0, int smem, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel<WARPS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    absa_sample_kernel<WARPS><<<(unsigned)rows, 32 * WARPS, smem, stream>>>(
+        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0, systematic);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
                           bool systematic, int cap, int32_t *counts, int32_t *kv_index,
                           float *log_pi, uint64_t *r_R, int32_t *status, int64_t row0,
@@ -435,12 +449,17 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
     const int ngroups = (nkb + 31) / 32;
     const int ngp = (ngroups + 7) & ~7;
     const int smem = (ngp * 32 + 2 * ngp + kCandMax) * 4;
-    cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    absa_sample_kernel<<<(unsigned)rows, kSampleThreads, smem, stream>>>(
-        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0, systematic);
-    return cudaGetLastError();
+    // The shared score copy limits the CTAs per SM (228 KB, 1 KB reserved
+    // per CTA); wider CTAs keep about 32 warps per SM when few CTAs fit.
+    const int per_sm = (228 * 1024) / (smem + 1024);
+    if (per_sm >= 4)
+        return launch_sample_w<8>(scores, rows, nkb, n, seed, systematic, cap, counts, kv_index,
+                                  log_pi, r_R, status, row0, smem, stream);
+    if (per_sm >= 2)
+        return launch_sample_w<16>(scores, rows, nkb, n, seed, systematic, cap, counts, kv_index,
+                                   log_pi, r_R, status, row0, smem, stream);
+    return launch_sample_w<32>(scores, rows, nkb, n, seed, systematic, cap, counts, kv_index,
+                               log_pi, r_R, status, row0, smem, stream);
 }
 
 }  // namespace absa
