@@ -34,6 +34,10 @@ struct Score2Smem {
     static constexpr int kTile = 128 * 128;                      // one region of 128 rows (bytes)
     static constexpr int kKeyTileBytes = 2 * kRegions * kTile;   // hi + lo of 128 key blocks
     static constexpr int kMuTileBytes = kRegions * kTile;        // 128 centroid rows (hi)
+    // key blocks of the range: [hi | lo][region][256 rows] (region r of both
+    // key tiles contiguous, so that one MMA can take all 256 rows as N)
+    static constexpr int kKeyRegion = kScoreKeyTiles * kTile;    // 256 rows of one region
+    static constexpr int kKeyLoOff = kRegions * kKeyRegion;      // lo parts after the hi parts
     static constexpr int kKeyOff = 0;
     static constexpr int kMuOff = kScoreKeyTiles * kKeyTileBytes;  // 2-stage centroid ring
     static constexpr int kXOff = kMuOff + 2 * kMuTileBytes;      // f32 [2][2][128] half exchange
@@ -105,14 +109,14 @@ struct ScoreCta {
                             int32_t *status) {
         tma_prefetch_desc(tm_mu_hi);
         mbar_arrive_expect_tx(key_full, kScoreKeyTiles * S::kKeyTileBytes);
-        for (int kt = 0; kt < kScoreKeyTiles; ++kt) {
-            const uint32_t base = smem_u32(sm + S::kKeyOff + kt * S::kKeyTileBytes);
+        const uint32_t kbase = smem_u32(sm + S::kKeyOff);
+        for (int kt = 0; kt < kScoreKeyTiles; ++kt)
             for (int r = 0; r < S::kRegions; ++r) {
-                tma_load_2d(base + r * S::kTile, tm_kb_hi, 64 * r, key_row0 + 128 * kt, key_full);
-                tma_load_2d(base + (S::kRegions + r) * S::kTile, tm_kb_lo, 64 * r,
-                            key_row0 + 128 * kt, key_full);
+                const uint32_t off = r * S::kKeyRegion + kt * S::kTile;
+                tma_load_2d(kbase + off, tm_kb_hi, 64 * r, key_row0 + 128 * kt, key_full);
+                tma_load_2d(kbase + S::kKeyLoOff + off, tm_kb_lo, 64 * r, key_row0 + 128 * kt,
+                            key_full);
             }
-        }
         for (int m = 0; m < nmt; ++m) {
             const int st = m & 1;
             if (m >= 2 && !mbar_wait(mu_empty + st, ((m - 2) >> 1) & 1, status, abort_flag)) break;
@@ -125,9 +129,10 @@ struct ScoreCta {
 
     // warp 1, one thread
     __device__ void mma(uint32_t tmem, int nmt, int32_t *status) {
-        constexpr uint32_t idesc = idesc_f16_f32(128, 128, 0);
-        constexpr uint32_t lo = S::kRegions * S::kTile;  // a key tile's lo part
+        constexpr uint32_t idesc128 = idesc_f16_f32(128, 128, 0);
+        constexpr uint32_t idesc256 = idesc_f16_f32(128, 256, 0);
         if (!mbar_wait(key_full, 0, status, abort_flag)) return;
+        const uint32_t kbase = smem_u32(sm + S::kKeyOff);
         for (int m = 0; m < nmt; ++m) {
             const int st = m & 1, buf = m & 1;
             if (!mbar_wait(mu_full + st, (m >> 1) & 1, status, abort_flag)) return;
@@ -135,23 +140,32 @@ struct ScoreCta {
                 return;
             tc_fence_after();
             const uint32_t mu_base = smem_u32(sm + S::kMuOff + st * S::kMuTileBytes);
+            if (TRANSPOSED) {
+                // D[key, centroid] per key tile: A = 128 key rows (hi, then lo), B = centroids
 #pragma unroll
-            for (int kt = 0; kt < kScoreKeyTiles; ++kt) {
-                const uint32_t key_base = smem_u32(sm + S::kKeyOff + kt * S::kKeyTileBytes);
-                const uint32_t dt = tmem + buf * 256 + kt * 128;
+                for (int kt = 0; kt < kScoreKeyTiles; ++kt) {
+                    const uint32_t dt = tmem + buf * 256 + kt * 128;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t koff = (ks >> 2) * S::kKeyRegion + kt * S::kTile + (ks & 3) * 32;
+                        const uint32_t moff = (ks >> 2) * S::kTile + (ks & 3) * 32;
+                        const uint64_t mu_d = sw128_desc(mu_base + moff, 16, 1024);
+                        tc_mma_f16(dt, sw128_desc(kbase + koff, 16, 1024), mu_d, idesc128, ks > 0);
+                        tc_mma_f16(dt, sw128_desc(kbase + S::kKeyLoOff + koff, 16, 1024), mu_d,
+                                   idesc128, 1);
+                    }
+                }
+            } else {
+                // D[centroid, key] for all 256 key blocks at once: N = 256
+                const uint32_t dt = tmem + buf * 256;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
-                    const uint64_t mu_d = sw128_desc(mu_base + off, 16, 1024);
-                    const uint64_t kh = sw128_desc(key_base + off, 16, 1024);
-                    const uint64_t kl = sw128_desc(key_base + lo + off, 16, 1024);
-                    if (TRANSPOSED) {
-                        tc_mma_f16(dt, kh, mu_d, idesc, ks > 0);
-                        tc_mma_f16(dt, kl, mu_d, idesc, 1);
-                    } else {
-                        tc_mma_f16(dt, mu_d, kh, idesc, ks > 0);
-                        tc_mma_f16(dt, mu_d, kl, idesc, 1);
-                    }
+                    const uint32_t koff = (ks >> 2) * S::kKeyRegion + (ks & 3) * 32;
+                    const uint32_t moff = (ks >> 2) * S::kTile + (ks & 3) * 32;
+                    const uint64_t mu_d = sw128_desc(mu_base + moff, 16, 1024);
+                    tc_mma_f16(dt, mu_d, sw128_desc(kbase + koff, 16, 1024), idesc256, ks > 0);
+                    tc_mma_f16(dt, mu_d, sw128_desc(kbase + S::kKeyLoOff + koff, 16, 1024),
+                               idesc256, 1);
                 }
             }
             tc_commit(d_full + buf);
