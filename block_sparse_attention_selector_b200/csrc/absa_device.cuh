@@ -47,25 +47,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-// Raise the expected transaction bytes of the current phase (no arrival).
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // try_wait with a suspend-time hint: the thread sleeps until the phase
 // completes or about `hint_ns` nanoseconds pass, without spinning.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
@@ -81,11 +62,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
     return ok != 0;
 }
 
-// Wait for the phase with the given parity.  Returns false (after setting the
-// timeout flag in *status and *abort) if it does not complete within about
-// kWaitLimitCycles, or if another thread of the CTA already gave up.  After a
-// short poll the thread sleeps between checks; the clock and the abort flag
-// are read once every 16 sleeps so that waiting warps take few issue slots.
+// Non-blocking test of the phase with the given parity.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -98,6 +75,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Wait for the phase with the given parity.  Returns false (after setting the
+// timeout flag in *status and *abort) if it does not complete within about
+// kWaitLimitCycles, or if another thread of the CTA already gave up.  After a
+// short poll the thread sleeps between checks; the clock and the abort flag
+// are read once every 16 sleeps so that waiting warps take few issue slots.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
                                           volatile int *abort) {
     // short non-blocking poll first: most waits end within a few hundred cycles
@@ -116,28 +98,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
             }
         }
     }
-}
-
-// ------------------------------------------------------------------ cp.async
-
-// 16-byte global->shared copy; src_bytes = 0 writes zeros without reading.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed
-// (the pending count is raised now and lowered on completion, so the thread
-// also makes its own regular arrive).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
