@@ -242,6 +242,23 @@ def recorded_traffic(kernel_src, w):
     return None
 
 
+def max_over_ranks(value, device, world):
+    """The largest `value` over the ranks: a collective that every rank calls
+    (with world == 1 it returns the value)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def per_call_ms(t_max_ms, steps, world):
+    """ms per call over the job: `world` ranks ran `steps` calls each within t_max_ms."""
+    return t_max_ms / (steps * world)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -318,11 +335,8 @@ def run_ours(args):
     att = np.array([e[2].elapsed_time(e[3]) for e in events])
     tot = sel + smp + att
     t_local = float(tot.sum())
-    t = torch.tensor([t_local], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    t_max = float(t.item())
-    ms_per_call = t_max / (K * world)
+    t_max = max_over_ranks(t_local, dev, world)
+    ms_per_call = per_call_ms(t_max, K, world)
 
     # dense reference kernel on the same shapes (companion number)
     ev_d = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -355,10 +369,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         if i > 0:
             e2e.append(e0.elapsed_time(e1))
-    te = torch.tensor([float(np.sum(e2e))], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / (max(1, len(e2e)) * world) if e2e else None
+    te_max = max_over_ranks(float(np.sum(e2e)), dev, world)
+    e2e_ms = per_call_ms(te_max, max(1, len(e2e)), world) if e2e else None
 
     burst_tf, sustained_tf, hbm_gbs, peak_src = measured_peaks()
     clk = clocks.summary()
