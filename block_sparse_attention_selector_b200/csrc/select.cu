@@ -121,9 +121,10 @@ __global__ void __launch_bounds__(128, 5) absa_kmeans_kernel(
     }
     {
         // K1: pooled keys of the same 128-token range, key blocks 32 qb .. 32 qb + 31,
-        // two chunks per thread at a time with all their loads issued first
+        // one chunk per thread at a time with its four loads issued first (two at a
+        // time spill at the 96 registers of five CTAs per SM)
         constexpr int UPT = CPR / 4;  // 32 blocks x CPR chunks over 128 threads
-        constexpr int BATCH = UPT < 2 ? UPT : 2;
+        constexpr int BATCH = 1;
         const int jb0 = qb * 32;
         const int nblk = min(32, nkb - jb0);
         const __nv_bfloat16 *ksrc = k + (bh * N + (int64_t)qb * 128) * D;
