@@ -50,8 +50,9 @@ def parse():
     ap.add_argument("--workload", default="wan480", choices=WORKLOADS,
                     help="layer to time: Wan2.1 480p (the default and the headline), Wan2.1 720p "
                          "or HunyuanVideo 720p")
-    ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic"],
-                    help="SIP design: Poisson draws (default) or systematic (exactly n blocks)")
+    ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic", "paired"],
+                    help="SIP design: Poisson draws (default), systematic (exactly n blocks) or "
+                         "paired (Poisson draws shared by query blocks 2p and 2p+1)")
     ap.add_argument("--harness", action="store_true",
                     help="mass-retention / error harness on the 480p and 720p layers (JSON lines; "
                          "no main line)")

@@ -29,14 +29,16 @@ def version():
     return _abi.version()
 
 
-SAMPLING = {"poisson": _abi.ABSA_SAMPLING_POISSON, "systematic": _abi.ABSA_SAMPLING_SYSTEMATIC}
+SAMPLING = {"poisson": _abi.ABSA_SAMPLING_POISSON, "systematic": _abi.ABSA_SAMPLING_SYSTEMATIC,
+            "paired": _abi.ABSA_SAMPLING_PAIRED}
 
 
 def make_params(B, H, N, d, T, Hg, Wg, budget_blocks, seed=0, softmax_scale=None,
                 kmeans_iters=3, sampling="poisson"):
     """An absa_params block (q_block 128, kv_block 4, 8 clusters).
 
-    sampling: "poisson" (independent draws) or "systematic" (exactly budget_blocks blocks)."""
+    sampling: "poisson" (independent draws), "systematic" (exactly budget_blocks
+    blocks) or "paired" (Poisson draws shared by query blocks 2p and 2p+1)."""
     p = absa_params()
     p.B, p.H, p.N, p.d = int(B), int(H), int(N), int(d)
     p.T, p.Hg, p.Wg = int(T), int(Hg), int(Wg)

@@ -33,6 +33,7 @@ EXPORTED = (
 ABSA_STATIC_SCRATCH_BYTES = 64 << 20
 ABSA_SAMPLING_POISSON = 0
 ABSA_SAMPLING_SYSTEMATIC = 1
+ABSA_SAMPLING_PAIRED = 2
 
 
 class absa_params(ctypes.Structure):

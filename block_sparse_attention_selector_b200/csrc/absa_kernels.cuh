@@ -27,10 +27,10 @@ cudaError_t launch_score(const CUtensorMap &tm_kb_hi, const CUtensorMap &tm_kb_l
                          float *part_s, float *L, float *scores, int64_t BH, int nqb, int nkb,
                          int d, float softmax_scale, int32_t *status, cudaStream_t stream);
 
-// K4: SIP plan rows from a score array.
+// K4: SIP plan rows from a score array.  design is an ABSA_SAMPLING_* value;
+// nqb (query blocks per head) places each global row in its query-block pair.
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
-                          bool systematic,
-                          int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
+                          int design, int nqb, int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
                           uint64_t *r_R, int32_t *status, int64_t row0, cudaStream_t stream);
 
 // K5 (dense = false) / K6 (dense = true): attention over 128-token tiles.

@@ -147,7 +147,8 @@ absa_status absa_check_params(const absa_params *p) {
     if (p->budget_blocks < 1 || p->kmeans_iters < 1 || p->kmeans_iters > 16)
         return ABSA_ERR_INVALID_ARG;
     if (!isfinite(p->softmax_scale)) return ABSA_ERR_INVALID_ARG;
-    if (p->sampling != ABSA_SAMPLING_POISSON && p->sampling != ABSA_SAMPLING_SYSTEMATIC)
+    if (p->sampling != ABSA_SAMPLING_POISSON && p->sampling != ABSA_SAMPLING_SYSTEMATIC &&
+        p->sampling != ABSA_SAMPLING_PAIRED)
         return ABSA_ERR_INVALID_ARG;
     if (p->q_block != 128 || p->kv_block != 4 || p->n_clusters != 8) return ABSA_ERR_UNSUPPORTED;
     if (p->d != 64 && p->d != 128) return ABSA_ERR_UNSUPPORTED;
@@ -235,7 +236,7 @@ absa_status sample_plan_run(const absa_params *p, const float *scores, const abs
     const int64_t row0 = hr.bh0 * dm.nqb, cap = plan->capacity;
     return from_cuda(launch_sample(scores + row0 * dm.nkb, hr.nbh * dm.nqb, dm.nkb,
                                    p->budget_blocks, p->seed,
-                                   p->sampling == ABSA_SAMPLING_SYSTEMATIC, plan->capacity,
+                                   p->sampling, dm.nqb, plan->capacity,
                                    plan->counts + row0,
                                    plan->kv_index + row0 * cap, plan->log_pi + row0 * cap,
                                    plan->r_R + 2 * row0, plan->status, row0, s));

@@ -10,7 +10,9 @@
 // same plan): q_j = max(1, floor(s_j 2^32)); capping fixed point on
 // (r, R) = (n - |C|, sum_{j not in C} q_j) with u64 block reductions; draw
 // u_j * R < (r q_j) 2^32 compared exactly.  u_j is output ctr+1 of the
-// SplitMix64 generator started from state mix(seed), ctr = row * NKB + j.
+// SplitMix64 generator started from state mix(seed), ctr = row * NKB + j;
+// the paired design draws query blocks 2p and 2p+1 of a head from the
+// counters of block 2p, so their samples nest block by block.
 #include "absa_kernels.cuh"
 
 namespace absa {
@@ -107,7 +109,7 @@ template <int WARPS>
 __global__ void __launch_bounds__(32 * WARPS) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
-    uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, bool systematic) {
+    uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, int design, int nqb) {
     constexpr int kSampleWarps = WARPS;
     constexpr int kSampleThreads = 32 * WARPS;
     extern __shared__ __align__(16) uint32_t samp_smem[];
@@ -289,13 +291,16 @@ __global__ void __launch_bounds__(32 * WARPS) absa_sample_kernel(
     const uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
 
     // SplitMix64 state of block j is base + j * gamma with
-    // base = mix(seed) + (global row * NKB + 1) * gamma
-    const uint64_t base =
-        splitmix64_mix(seed) + ((uint64_t)(row0 + row) * (uint64_t)nkb + 1) * kGamma;
+    // base = mix(seed) + (draw row * NKB + 1) * gamma; the draw row is the
+    // global row, or under the paired design that of the even query block of
+    // the pair (qb with its low bit cleared)
+    const int64_t grow = row0 + row;
+    const int64_t drow = design == ABSA_SAMPLING_PAIRED ? grow - ((grow % nqb) & 1) : grow;
+    const uint64_t base = splitmix64_mix(seed) + ((uint64_t)drow * (uint64_t)nkb + 1) * kGamma;
     const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
     int taken = 0;
-    if (!systematic) {
-        // Poisson draws: one taken word per group
+    if (design != ABSA_SAMPLING_SYSTEMATIC) {
+        // Poisson draws (own or paired counters): one taken word per group
         uint64_t state = base + (uint64_t)(g0 * 32 + lane) * kGamma;  // state of block j
         for (int g = g0; g < g1; ++g, state += 32 * kGamma) {
             const int j = g * 32 + lane;
@@ -431,19 +436,19 @@ __global__ void __launch_bounds__(32 * WARPS) absa_sample_kernel(
 
 template <int WARPS>
 static cudaError_t launch_sample_w(const float *scores, int64_t rows, int nkb, int64_t n,
-                                   uint64_t seed, bool systematic, int cap, int32_t *counts,
+                                   uint64_t seed, int design, int nqb, int cap, int32_t *counts,
                                    int32_t *kv_index, float *log_pi, uint64_t *r_R,
                                    int32_t *status, int64_t row0, int smem, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel<WARPS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     absa_sample_kernel<WARPS><<<(unsigned)rows, 32 * WARPS, smem, stream>>>(
-        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0, systematic);
+        scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0, design, nqb);
     return cudaGetLastError();
 }
 
 cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n, uint64_t seed,
-                          bool systematic, int cap, int32_t *counts, int32_t *kv_index,
+                          int design, int nqb, int cap, int32_t *counts, int32_t *kv_index,
                           float *log_pi, uint64_t *r_R, int32_t *status, int64_t row0,
                           cudaStream_t stream) {
     const int ngroups = (nkb + 31) / 32;
@@ -453,12 +458,12 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
     // per CTA); wider CTAs keep about 32 warps per SM when few CTAs fit.
     const int per_sm = (228 * 1024) / (smem + 1024);
     if (per_sm >= 4)
-        return launch_sample_w<8>(scores, rows, nkb, n, seed, systematic, cap, counts, kv_index,
+        return launch_sample_w<8>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
                                   log_pi, r_R, status, row0, smem, stream);
     if (per_sm >= 2)
-        return launch_sample_w<16>(scores, rows, nkb, n, seed, systematic, cap, counts, kv_index,
+        return launch_sample_w<16>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
                                    log_pi, r_R, status, row0, smem, stream);
-    return launch_sample_w<32>(scores, rows, nkb, n, seed, systematic, cap, counts, kv_index,
+    return launch_sample_w<32>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
                                log_pi, r_R, status, row0, smem, stream);
 }
 

@@ -107,6 +107,28 @@ def rel_l2(a, b):
     return float((a - b).norm() / b.norm())
 
 
+def pair_union_ratio(plan, nkb):
+    """Blocks in the union of the samples of query blocks 2p and 2p+1, over
+    the blocks the two samples hold: what a kernel loading each pair's union
+    once would compute per query block (1 when the samples coincide, 2 when
+    they are disjoint)."""
+    import torch
+
+    cnt = plan.counts
+    B, H, nqb = cnt.shape
+    npair = nqb // 2
+    if npair == 0:
+        return math.nan
+    taken = torch.zeros(B, H, 2 * npair, nkb + 1, dtype=torch.bool, device=cnt.device)
+    cap = plan.kv_index.shape[-1]
+    valid = torch.arange(cap, device=cnt.device) < cnt[..., None]
+    idx = torch.where(valid, plan.kv_index.long(), nkb)[:, :, :2 * npair]
+    taken.scatter_(-1, idx, True)
+    taken = taken[..., :nkb].reshape(B, H, npair, 2, nkb)
+    union = (taken[:, :, :, 0] | taken[:, :, :, 1]).sum()
+    return float(2 * union) / float(taken.sum())
+
+
 def retention_report(w, q, k, v, budget=None, seed=0):
     """One layer: retained mass and relative L2 error of every selector at n blocks."""
     import torch
@@ -138,12 +160,14 @@ def retention_report(w, q, k, v, budget=None, seed=0):
                                                    .sum(dim=-1).mean())
     out["blocks_128token"] = n128
 
-    for design in ("poisson", "systematic"):
+    for design in ("poisson", "systematic", "paired"):
         ps = params_for(w, seed=seed, budget=n, sampling=design)
         plan = sample_plan(ps, scores)
         plan.check()
         out[f"mass_sip_{design}"] = retained_mass(M, plan.kv_index, plan.counts)
         out[f"mean_blocks_sip_{design}"] = float(plan.counts.float().mean())
+        if design != "systematic":
+            out[f"pair_union_over_own_{design}"] = pair_union_ratio(plan, nkb)
         o = sparse_attention(ps, q, k, v, plan)
         out[f"rel_l2_sip_{design}"] = rel_l2(o, o_dense)
 

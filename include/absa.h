@@ -64,13 +64,15 @@ typedef struct {
     int32_t budget_blocks;  /* n: expected KV blocks per query block; n >= NKB = dense */
     uint64_t seed;          /* SIP draw seed                                          */
     float softmax_scale;    /* logit scale, normally 1/sqrt(d)                        */
-    int32_t sampling;       /* SIP design: ABSA_SAMPLING_POISSON (0, the default) or  */
-                            /* ABSA_SAMPLING_SYSTEMATIC (1); see absa_sample_plan     */
+    int32_t sampling;       /* SIP design: ABSA_SAMPLING_POISSON (0, the default),    */
+                            /* ABSA_SAMPLING_SYSTEMATIC (1) or ABSA_SAMPLING_PAIRED   */
+                            /* (2); see absa_sample_plan                              */
 } absa_params;
 
 /* Sampling designs of the SIP sampler (absa_params.sampling). */
 #define ABSA_SAMPLING_POISSON 0
 #define ABSA_SAMPLING_SYSTEMATIC 1
+#define ABSA_SAMPLING_PAIRED 2
 
 typedef struct {
     /* All arrays are caller-owned device memory sized from absa_plan_capacity. */
@@ -151,6 +153,14 @@ absa_status absa_select_scores(const absa_params *p, const void *q, const void *
  *    U = u(row*NKB), points sit at (k + U/2^32)*R for k = 0..n-1 and block j
  *    is taken iff a point falls in [sum_{i<j} a_i, sum_{i<=j} a_i).  Every
  *    block is taken with probability pi_j and exactly n blocks are taken.
+ *  - ABSA_SAMPLING_PAIRED: the Poisson rule with the draws of query block
+ *    qb & ~1 of the same (b,h): block j of row (b,h,qb) is taken iff j in C
+ *    or u(row'*NKB + j) * R < r*q_j * 2^32, row' = (b*H + h)*NQB + (qb & ~1).
+ *    Each row is still a Poisson sample with its own pi; the two rows of a
+ *    pair share one uniform per block, so the row with the smaller pi_j
+ *    takes j only if the other does (their samples nest block by block and
+ *    their union has expected size sum_j max(pi_0j, pi_1j)).  A last query
+ *    block without a partner (NQB odd) keeps its own draws.
  * Taken blocks are written ascending
  * with log_pi = 0 (capped) or (float)ln((double)(r*q_j)/R).  n >= NKB takes
  * every block.  Resets plan->status first; a row with more than

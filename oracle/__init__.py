@@ -235,8 +235,9 @@ def systematic_take(s, n, U):
 def sample_plan(scores, n, seed, cap, design="poisson"):
     """SIP plan for every row of a [B,H,NQB,NKB] fp32 score array.
 
-    design: "poisson" or "systematic".  Returns dict(counts, kv_index, log_pi, r_R,
-    overflow_rows).
+    design: "poisson", "systematic" or "paired" (Poisson draws shared by the
+    query blocks 2p and 2p+1 of a head).  Returns dict(counts, kv_index, log_pi,
+    r_R, overflow_rows).
     """
     scores = _c(scores, np.float32)
     B, H, nqb, nkb = scores.shape
@@ -246,7 +247,7 @@ def sample_plan(scores, n, seed, cap, design="poisson"):
     r_R = np.zeros((B, H, nqb, 2), np.uint64)
     ov = lib().oracle_sample_plan_design(B, H, nqb, nkb, int(n), int(seed), scores, int(cap),
                                          counts, idx, lp, r_R,
-                                         {"poisson": 0, "systematic": 1}[design])
+                                         {"poisson": 0, "systematic": 1, "paired": 2}[design])
     return dict(counts=counts, kv_index=idx, log_pi=lp, r_R=r_R, overflow_rows=int(ov))
 
 

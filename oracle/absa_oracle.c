@@ -471,15 +471,18 @@ void oracle_select_scores(int B, int H, int64_t N, int d, int nc, int iters,
 int oracle_sample_plan_design(int B, int H, int nqb, int nkb, int64_t n,
                               uint64_t seed, const float *scores, int cap,
                               int32_t *counts, int32_t *kv_index, float *log_pi,
-                              uint64_t *r_R, int systematic)
+                              uint64_t *r_R, int design)
 {
     int overflow = 0;
     int64_t rows = (int64_t)B * H * nqb;
 #pragma omp parallel for schedule(dynamic, 16) reduction(+ : overflow)
     for (int64_t row = 0; row < rows; ++row) {
         uint64_t r, R;
-        int taken = (systematic ? oracle_sample_row_systematic : oracle_sample_row)(
-            scores + row * nkb, nkb, n, seed, (uint64_t)row, cap, kv_index + row * cap,
+        /* paired design: the draws of row (b,h,qb) are those of (b,h,qb with
+         * its low bit cleared) */
+        const int64_t draw_row = design == 2 ? row - ((row % nqb) & 1) : row;
+        int taken = (design == 1 ? oracle_sample_row_systematic : oracle_sample_row)(
+            scores + row * nkb, nkb, n, seed, (uint64_t)draw_row, cap, kv_index + row * cap,
             log_pi + row * cap, &r, &R);
         counts[row] = taken < cap ? taken : cap;
         r_R[2 * row] = r;

@@ -155,12 +155,20 @@ int oracle_sample_plan(int B, int H, int nqb, int nkb, int64_t n,
                        int32_t *counts, int32_t *kv_index, float *log_pi,
                        uint64_t *r_R);
 
-/* oracle_sample_plan with the design chosen: systematic = 0 Poisson,
- * 1 systematic (oracle_sample_row_systematic). */
+/* oracle_sample_plan with the design chosen: 0 Poisson, 1 systematic
+ * (oracle_sample_row_systematic), 2 paired Poisson.  Paired: the Poisson
+ * design whose draws for query block qb are those of query block
+ * qb & ~1 of the same (b,h) (counter row ((b*H + h)*NQB + (qb & ~1))), so the
+ * two query blocks of a pair share one uniform per KV block.  Each row is
+ * still a Poisson sample with its own pi (the Horvitz-Thompson estimate of
+ * every row stays unbiased); across a pair, block j is in the sample with the
+ * smaller pi_j only if it is in the other (the samples nest block by block),
+ * so their union has expected size sum_j max(pi_0j, pi_1j).  A last query
+ * block without a partner (NQB odd) keeps its own draws. */
 int oracle_sample_plan_design(int B, int H, int nqb, int nkb, int64_t n,
                               uint64_t seed, const float *scores, int cap,
                               int32_t *counts, int32_t *kv_index, float *log_pi,
-                              uint64_t *r_R, int systematic);
+                              uint64_t *r_R, int design);
 
 /* HT sparse attention for every valid query row of query blocks
  * qb_lo <= qb < qb_hi with the given plan.  o is [B,H,N,d] fp64; rows

@@ -76,7 +76,7 @@ def test_workspace_bytes_covers_layout(L):
     ("budget_blocks", 0, _abi.ABSA_ERR_INVALID_ARG),
     ("kmeans_iters", 0, _abi.ABSA_ERR_INVALID_ARG),
     ("softmax_scale", float("nan"), _abi.ABSA_ERR_INVALID_ARG),
-    ("sampling", 2, _abi.ABSA_ERR_INVALID_ARG),
+    ("sampling", 3, _abi.ABSA_ERR_INVALID_ARG),
     ("sampling", -1, _abi.ABSA_ERR_INVALID_ARG),
 ])
 def test_bad_params_rejected(L, field, value, code):
@@ -129,9 +129,9 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 
 def test_params_struct_matches_the_header(L):
     # the Python mirror of absa_params has the C layout: 12 int32, u64 seed, float scale,
-    # int32 sampling (64 bytes); both sampling designs validate
+    # int32 sampling (64 bytes); every sampling design validates
     assert ctypes.sizeof(_abi.absa_params) == 64
     assert _abi.absa_params.sampling.offset == 60
-    for design in ("poisson", "systematic"):
+    for design in ("poisson", "systematic", "paired"):
         p = make_params(1, 2, 512, 64, 4, 8, 16, 13, sampling=design)
         assert _abi.absa_check_params(p) == _abi.ABSA_OK

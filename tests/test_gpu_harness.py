@@ -63,10 +63,14 @@ def test_retention_report_invariants(w):
     assert rep["mean_blocks_sip_systematic"] == w.budget
     assert 0.0 < rep["mass_ideal_topk_128token_blocks"] <= 1.0 + 1e-2
     assert abs(rep["mass_row_sum_mean"] - 1.0) < 1e-2
+    # shared draws make the two samples of a query-block pair overlap more
+    assert 1.0 <= rep["pair_union_over_own_paired"] < rep["pair_union_over_own_poisson"] <= 2.0
     # every key block: all selectors keep everything and reproduce dense attention
     full, _ = harness.retention_report(w, qd, kd, vd, budget=w.nkb, seed=3)
     for key in ("mass_ideal_topk", "mass_block_mean", "mass_ibcs_topn", "mass_sip_poisson",
-                "mass_sip_systematic"):
+                "mass_sip_systematic", "mass_sip_paired"):
         assert abs(full[key] - 1.0) < 1e-2, (key, full[key])
-    for key in ("rel_l2_ideal_topk", "rel_l2_sip_poisson", "rel_l2_sip_systematic"):
+    for key in ("rel_l2_ideal_topk", "rel_l2_sip_poisson", "rel_l2_sip_systematic",
+                "rel_l2_sip_paired"):
         assert full[key] == 0.0, (key, full[key])
+    assert full["pair_union_over_own_paired"] == 1.0

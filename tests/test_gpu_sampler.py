@@ -21,7 +21,8 @@ def _params(nkb, rows_h, n, seed, sampling="poisson"):
 
 
 def _compare(p, scores, plan_gpu, cap):
-    design = "systematic" if p.sampling == _abi.ABSA_SAMPLING_SYSTEMATIC else "poisson"
+    design = {_abi.ABSA_SAMPLING_POISSON: "poisson", _abi.ABSA_SAMPLING_SYSTEMATIC: "systematic",
+              _abi.ABSA_SAMPLING_PAIRED: "paired"}[p.sampling]
     ref = oracle.sample_plan(scores, p.budget_blocks, p.seed, cap, design=design)
     got = plan_to_numpy(plan_gpu)
     assert np.array_equal(got["counts"], ref["counts"])
@@ -156,3 +157,57 @@ def test_systematic_full_layer_plan_and_attention():
                                                  ref["log_pi"][0, h, qb, :c], 1 / math.sqrt(w.d))
             mx, rel = attention_errors(o[0, h, rows].float().cpu().numpy(), o_ref)
             assert mx <= ATTN_MAX_ABS and rel <= ATTN_REL_L2, (h, qb, mx, rel)
+
+
+# The paired design (query blocks 2p and 2p+1 share their draws): same bar, on
+# layouts with an even and an odd number of query blocks per head (the last
+# block of an odd head draws alone) and several heads.
+@pytest.mark.parametrize("nkb,H,n,seed", [(128, 3, 13, 0), (515, 3, 40, 1), (1000, 2, 100, 2),
+                                          (8190, 2, 819, 3), (515, 2, 514, 4)])
+def test_paired_sampler_bit_exact_on_identical_scores(nkb, H, n, seed):
+    import torch
+
+    p = _params(nkb, H, n, seed, sampling="paired")
+    nqb = (p.N + 127) // 128
+    scores = synthetic.random_scores(H * nqb, nkb, seed, concentration=1.0).reshape(1, H, nqb,
+                                                                                    nkb)
+    plan = sample_plan(p, torch.from_numpy(scores).cuda())
+    plan.check()
+    _compare(p, scores, plan, plan.capacity)
+
+
+def test_paired_full_layer_plans_nest():
+    """select_plan with the paired design on the Wan2.1 480p layer cut to 4
+    heads: the plan bit-equal to the oracle's from the GPU's own scores, and
+    within every query-block pair the row with the smaller pi_j takes block j
+    only if its partner does."""
+    import dataclasses
+
+    import torch
+    from block_sparse_attention_selector_b200 import params_for, select_plan
+    from gpu_helpers import device_bf16
+
+    w = dataclasses.replace(synthetic.WAN480, H=4)
+    q, k, _ = synthetic.layer_qkv_bits(w)
+    p = params_for(w, seed=3, sampling="paired")
+    plan, scores, _ = select_plan(p, device_bf16(q), device_bf16(k))
+    plan.check()
+    s = scores.cpu().numpy()
+    ref = _compare(p, s, plan, plan.capacity)
+    for h in (0, w.H - 1):
+        for qb in range(0, w.nqb - 1, 18):  # every ninth pair
+            takes = []
+            pis = []
+            for r in (qb, qb + 1):
+                t = np.zeros(w.nkb, bool)
+                t[ref["kv_index"][0, h, r, :ref["counts"][0, h, r]]] = True
+                takes.append(t)
+                capped, rr, RR, _ = oracle.pi_solve(s[0, h, r], w.budget)
+                qv = np.array(oracle.quantised_scores(s[0, h, r]), dtype=object)
+                pis.append(np.where(capped, RR, rr * qv))  # pi_j * R, exact integers
+                pis[-1] = (pis[-1], RR)
+            (a0, R0), (a1, R1) = pis
+            lo0 = np.array([x * R1 <= y * R0 for x, y in zip(a0, a1)])  # pi_0j <= pi_1j
+            t_lo = np.where(lo0, takes[0], takes[1])
+            t_hi = np.where(lo0, takes[1], takes[0])
+            assert not np.any(t_lo & ~t_hi), (h, qb)

@@ -252,3 +252,86 @@ def test_systematic_plan_row_and_layer():
     # n >= nkb: every block
     idx, lp, taken, r, R = oracle.sample_row(s[0], 300, seed, 0, 300, design="systematic")
     assert taken == 300 and np.array_equal(idx, np.arange(300)) and not lp.any()
+
+
+# ---------------------------------------------------------------- paired design
+# Correlated draws across a pair of query blocks: blocks 2p and 2p+1 of a head
+# share the uniform of every KV block, so each row is still its own Poisson
+# sample with probabilities pi (the SIP paragraph's unbiasedness holds row by
+# row) while the two samples nest: a block in the sample with the smaller
+# pi_j is in the other.  Pins: that coupling identity on every block, the
+# joint inclusion frequencies P(both) = min(pi_0, pi_1) and
+# P(either) = max(pi_0, pi_1) over 10^4 seeds, and the marginals of the odd row.
+
+def _pair_scores(nkb, seed):
+    """Two correlated score rows (neighbouring query blocks attend alike)."""
+    base = synthetic.random_scores(1, nkb, seed, concentration=1.5)[0].astype(np.float64)
+    noise = synthetic.random_scores(1, nkb, seed + 1, concentration=1.5)[0]
+    s1 = 0.7 * base + 0.3 * noise
+    return np.stack([base, s1 / s1.sum()]).astype(np.float32)
+
+
+def _pair_plan(s2, n, seed, design="paired"):
+    nkb = s2.shape[-1]
+    plan = oracle.sample_plan(s2.reshape(1, 1, 2, nkb), n, seed, nkb, design=design)
+    takes = np.zeros((2, nkb), bool)
+    for qb in range(2):
+        takes[qb, plan["kv_index"][0, 0, qb, :plan["counts"][0, 0, qb]]] = True
+    return takes, plan
+
+
+def test_paired_samples_nest_block_by_block():
+    nkb, n = 500, 60
+    s2 = _pair_scores(nkb, 31)
+    p0 = np.array(pis(s2[0], n)[0])
+    p1 = np.array(pis(s2[1], n)[0])
+    lo_is_0 = p0 <= p1
+    for seed in range(50):
+        takes, _ = _pair_plan(s2, n, seed)
+        t_lo = np.where(lo_is_0, takes[0], takes[1])
+        t_hi = np.where(lo_is_0, takes[1], takes[0])
+        assert not np.any(t_lo & ~t_hi), seed
+
+
+def test_paired_joint_inclusion_frequencies():
+    nkb, n, S = 64, 10, 10000
+    s2 = _pair_scores(nkb, 41)
+    p0 = np.array(pis(s2[0], n)[0])
+    p1 = np.array(pis(s2[1], n)[0])
+    both = np.zeros(nkb)
+    either = np.zeros(nkb)
+    odd = np.zeros(nkb)
+    union_sizes = np.zeros(S)
+    for seed in range(S):
+        takes, _ = _pair_plan(s2, n, seed)
+        both += takes[0] & takes[1]
+        either += takes[0] | takes[1]
+        odd += takes[1]
+        union_sizes[seed] = (takes[0] | takes[1]).sum()
+    for freq, p in ((both / S, np.minimum(p0, p1)), (either / S, np.maximum(p0, p1)),
+                    (odd / S, p1)):
+        sigma = np.sqrt(p * (1 - p) / S) + 1e-12
+        assert np.all(np.abs(freq - p) <= 5 * sigma + 1e-12)
+    pm = np.maximum(p0, p1)
+    assert abs(union_sizes.mean() - pm.sum()) <= 5 * math.sqrt(float((pm * (1 - pm)).sum()) / S)
+    # independent draws would give sum(p0 + p1 - p0 p1) blocks in the union
+    assert pm.sum() < (p0 + p1 - p0 * p1).sum() - 5 * math.sqrt(float((pm * (1 - pm)).sum()) / S)
+
+
+def test_paired_rows_and_unpaired_tail():
+    # even query blocks keep their own Poisson draws, odd ones take their
+    # partner's counter row; with NQB odd the last block keeps its own
+    nkb, n, seed, nqb = 300, 30, 5, 3
+    s = synthetic.random_scores(2 * nqb, nkb, 51).reshape(1, 2, nqb, nkb)
+    cap = oracle.plan_capacity(n, nkb)
+    got = oracle.sample_plan(s, n, seed, cap, design="paired")
+    for h in range(2):
+        for qb in range(nqb):
+            row = h * nqb + qb
+            draw_row = row - 1 if qb % 2 == 1 else row
+            idx, lp, taken, r, R = oracle.sample_row(s[0, h, qb], n, seed, draw_row, cap)
+            c = got["counts"][0, h, qb]
+            assert c == min(taken, cap)
+            assert np.array_equal(got["kv_index"][0, h, qb, :c], idx[:c])
+            assert np.array_equal(got["log_pi"][0, h, qb, :c], lp[:c])
+            assert tuple(got["r_R"][0, h, qb]) == (r, R)
