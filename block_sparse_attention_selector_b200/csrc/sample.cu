@@ -106,7 +106,7 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
 // overflows or the threshold falls below the half, the remaining rounds scan
 // every block.  Either way the rounds are exactly those of the definition.
 template <int WARPS>
-__global__ void __launch_bounds__(32 * WARPS) absa_sample_kernel(
+__global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 5 : WARPS == 16 ? 2 : 1) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
     uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, int design, int nqb) {
@@ -294,8 +294,9 @@ __global__ void __launch_bounds__(32 * WARPS) absa_sample_kernel(
     // base = mix(seed) + (draw row * NKB + 1) * gamma; the draw row is the
     // global row, or under the paired design that of the even query block of
     // the pair (qb with its low bit cleared)
-    const int64_t grow = row0 + row;
-    const int64_t drow = design == ABSA_SAMPLING_PAIRED ? grow - ((grow % nqb) & 1) : grow;
+    // (row0 is a multiple of NQB: launches start at a head boundary)
+    const int64_t drow =
+        row0 + row - (design == ABSA_SAMPLING_PAIRED ? (int)(blockIdx.x % (unsigned)nqb) & 1 : 0);
     const uint64_t base = splitmix64_mix(seed) + ((uint64_t)drow * (uint64_t)nkb + 1) * kGamma;
     const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
     int taken = 0;
