@@ -3,7 +3,9 @@
 Heads are independent in every stage and the draw counter uses the global
 plan row, so running the step in runs of heads must give bit-for-bit the
 scores, plan and output of absa_select_plan + absa_sparse_attention over the
-whole problem, for every run length, with pinned or pageable host memory.
+whole problem, for every run length, with pinned or pageable host memory, and
+for the paired draws too (a run starts at a head boundary, so query-block
+pairs never straddle two runs).
 The output is also checked against the oracle fed the GPU's plan.
 """
 import numpy as np
@@ -27,12 +29,13 @@ def _host(bits, pin):
     return t.pin_memory() if pin else t.clone()
 
 
+@pytest.mark.parametrize("sampling", ["poisson", "paired"])
 @pytest.mark.parametrize("w", [RAGGED128, HEADS5], ids=lambda w: w.name)
-def test_step_host_equals_device_calls(w):
+def test_step_host_equals_device_calls(w, sampling):
     import torch
 
     q, k, v = synthetic.layer_qkv_bits(w)
-    p = params_for(w, seed=23)
+    p = params_for(w, seed=23, sampling=sampling)
     qd, kd, vd = device_bf16(q), device_bf16(k), device_bf16(v)
     plan_ref, s_ref, _ = select_plan(p, qd, kd)
     o_ref = sparse_attention(p, qd, kd, vd, plan_ref)
