@@ -1,18 +1,21 @@
 """Benchmark of the AB-Attention hot path on B200.
 
-One step = one attention call of a Wan2.1-14B-shaped 480p self-attention layer
-(B=1, 40 heads, d=128, 21x30x52 = 32760 tokens, budget 819 of 8190 key blocks):
-IBCS selector (pool, k-means, score) + SIP sampler + HT sparse attention, all
-in libabsa.so.  Metric: ms per attention call (lower is better), with the
-effective TFLOP/s of the sparse attention beside it.
+One step = one attention call of a HunyuanVideo-shaped 720p self-attention
+layer by default (B=1, 24 heads, d=128, 33x45x80 = 118800 tokens, budget 2376
+of 29700 key blocks; --workload wan480 / wan720 select the Wan2.1-shaped
+layers): IBCS selector (pool + k-means, score) + SIP sampler + HT sparse
+attention, all in libabsa.so.  Metric: ms per attention call (lower is
+better), with the effective TFLOP/s of the sparse attention beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 N > 1 (under torchrun): every rank runs the same layer on its own GPU
 (independent replicas, no collective on the data path); the time is the max
-over ranks and the value is ms per call over all N*K calls.
+over ranks and the value is ms per call over all N*K calls (a throughput
+figure; per_gpu_ms beside it is the per-call latency of one GPU).
 --impl reference times the CPU oracle (plain C, OpenMP) on a bounded sample of
-the same layer and extrapolates to ms per call.
+the same layer (the first query blocks of every head) and extrapolates to ms
+per call; the line states the sampled work and the factor.
 """
 import argparse
 import hashlib
@@ -45,11 +48,11 @@ def parse():
                     help="target wall time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
-                    help="run only this many heads (profiling captures); 0 = all 40")
+                    help="run only this many heads (profiling captures); 0 = all heads of the layer")
     ap.add_argument("--dense-reps", type=int, default=3)
-    ap.add_argument("--workload", default="wan480", choices=WORKLOADS,
-                    help="layer to time: Wan2.1 480p (the default and the headline), Wan2.1 720p "
-                         "or HunyuanVideo 720p")
+    ap.add_argument("--workload", default="hunyuan720", choices=WORKLOADS,
+                    help="layer to time: HunyuanVideo 720p (the default and the headline: the "
+                         "largest single-GPU layer), Wan2.1 480p or Wan2.1 720p")
     ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic", "paired"],
                     help="SIP design: Poisson draws (default), systematic (exactly n blocks) or "
                          "paired (Poisson draws shared by query blocks 2p and 2p+1)")
@@ -67,7 +70,7 @@ def parse():
 WORKLOADS = ("wan480", "wan720", "hunyuan720")
 
 
-def workload(heads=0, name="wan480"):
+def workload(heads=0, name="hunyuan720"):
     from block_sparse_attention_selector_b200 import synthetic
 
     w = {"wan480": synthetic.WAN480, "wan720": synthetic.WAN720,
@@ -79,22 +82,21 @@ def workload(heads=0, name="wan480"):
     return w
 
 
-def config_of(w, extra=None, sampling="poisson"):
-    cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-           "grid": [w.T, w.Hg, w.Wg], "budget_blocks": w.budget, "sampling": sampling,
-           "kv_blocks": w.nkb,
-           "query_blocks": w.nqb, "inputs": "seeded synthetic Fourier-feature q/k, Gaussian v",
-           "l2": "flushed before every timed step (256 MiB write, outside the step events); "
-                 "inputs (1 GiB q/k/v) are also larger than L2"}
-    if extra:
-        cfg.update(extra)
-    return cfg
+def config_of(w, sampling="poisson"):
+    """The workload of a line (the same keys on both arms)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "grid": [w.T, w.Hg, w.Wg], "budget_blocks": w.budget, "sampling": sampling,
+            "kv_blocks": w.nkb,
+            "query_blocks": w.nqb, "inputs": "seeded synthetic Fourier-feature q/k, Gaussian v",
+            "l2": "flushed before every timed step (256 MiB write, outside the step events); "
+                  "inputs (q/k/v, 0.9-2.2 GiB) are also larger than L2"}
 
 
 # ------------------------------------------------------------------ CPU oracle
 
 def oracle_sample(w, q, k, v, n_qb, seed=1, design="poisson"):
-    """Run the oracle hot path on query blocks [0, n_qb) of every head; seconds."""
+    """Run the oracle hot path on query blocks [0, n_qb) of every head; seconds.  The
+    selector pools every head's keys whatever the range."""
     import oracle
 
     t0 = time.perf_counter()
@@ -112,17 +114,40 @@ def oracle_sample(w, q, k, v, n_qb, seed=1, design="poisson"):
     return time.perf_counter() - t0
 
 
+def oracle_pool_seconds(q, k):
+    """Oracle time of the per-head key pooling alone (an empty query-block range)."""
+    import oracle
+
+    t0 = time.perf_counter()
+    oracle.select_scores(q, k, qb_range=(1, 1))
+    return time.perf_counter() - t0
+
+
+def oracle_extrapolated_ms(w, t_step, t_pool, n_qb):
+    """ms per full-layer call from a sample of n_qb query blocks per head: the pooling
+    once, the per-query-block work scaled by NQB / n_qb."""
+    per_rows = max(t_step - t_pool, 0.0)
+    return (t_pool + per_rows * w.nqb / n_qb) * 1e3
+
+
+def oracle_sample_size(w, q, k, v, target_s, design):
+    t1 = oracle_sample(w, q, k, v, 1, design=design)
+    return int(max(1, min(w.nqb, math.floor(target_s / max(t1, 1e-3))))), t1
+
+
 def cpu_baseline(w, q, k, v, target_s, design="poisson"):
     import oracle
 
-    t1 = oracle_sample(w, q, k, v, 1, design=design)
-    n_qb = int(max(1, min(w.nqb, math.floor(target_s / max(t1, 1e-3)))))
+    n_qb, t1 = oracle_sample_size(w, q, k, v, target_s, design)
     t = oracle_sample(w, q, k, v, n_qb, design=design) if n_qb > 1 else t1
-    ms = t * 1e3 * w.nqb / n_qb
+    t_pool = oracle_pool_seconds(q, k)
+    ms = oracle_extrapolated_ms(w, t, t_pool, n_qb)
     return {"value": ms, "unit": "ms", "cores": oracle.num_threads(), "kind": "oracle",
+            "timed_query_blocks_per_head": n_qb, "extrapolation_factor": w.nqb / n_qb,
             "sample": f"query blocks 0..{n_qb - 1} of all {w.H} heads ({n_qb * w.H} of "
-                      f"{w.nqb * w.H} plan rows: select+sample+attention), wall {t:.1f} s, "
-                      f"extrapolated x{w.nqb / n_qb:.1f} to the full layer"}
+                      f"{w.nqb * w.H} plan rows: select+sample+attention) in {t:.1f} s, of which "
+                      f"{t_pool:.1f} s is the per-head key pooling; the rest is scaled "
+                      f"x{w.nqb / n_qb:.1f} to the full layer"}
 
 
 def run_reference(args):
@@ -138,18 +163,25 @@ def run_reference(args):
     oracle.lib()
     steps = max(1, args.steps)
     per_step_target = max(1.0, min(args.cpu_seconds, 120.0 / (steps + args.warmup)))
-    t1 = oracle_sample(w, q, k, v, 1, design=args.sampling)
-    n_qb = int(max(1, min(w.nqb, math.floor(per_step_target / max(t1, 1e-3)))))
+    n_qb, _ = oracle_sample_size(w, q, k, v, per_step_target, args.sampling)
+    t_pool = oracle_pool_seconds(q, k)
     for _ in range(args.warmup):
         oracle_sample(w, q, k, v, n_qb, design=args.sampling)
     times = [oracle_sample(w, q, k, v, n_qb, design=args.sampling) for _ in range(steps)]
-    ms = float(np.mean(times)) * 1e3 * w.nqb / n_qb
+    t_step = float(np.mean(times))
+    ms = oracle_extrapolated_ms(w, t_step, t_pool, n_qb)
     sample = (f"each step: query blocks 0..{n_qb - 1} of all {w.H} heads "
-              f"(select+sample+attention), extrapolated x{w.nqb / n_qb:.1f}")
+              f"(select+sample+attention, {t_step:.1f} s, of which {t_pool:.1f} s is the "
+              f"per-head key pooling); the rest is scaled x{w.nqb / n_qb:.1f} to the full layer")
     line = {"impl": "reference", "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": args.gpus,
-            "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, sampling=args.sampling),
+            # ms_per_step is the measured wall time of one sampled step (steps x ms_per_step
+            # is the timed run); value is the full-layer estimate from it
+            "steps": steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, sampling=args.sampling),
+            "sampled_work": {"timed_query_blocks_per_head": n_qb, "query_blocks_per_head": w.nqb,
+                             "heads": w.B * w.H, "extrapolation_factor": w.nqb / n_qb,
+                             "pool_seconds": t_pool, "step_seconds": t_step},
             "cpu_baseline": {"value": ms, "unit": "ms", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -243,6 +275,38 @@ def recorded_traffic(kernel_src, w):
     return None
 
 
+def selector_sampler_roofline(w, counts, kmeans_ms, score_ms, sample_ms, hbm_gbs, peak_src):
+    """HBM roofline of the selector + sampler (S2-S6).  Algorithmic bytes: read q and k
+    once, write the plan (kv_index + log_pi of every taken block, counts, r*/R*).  The
+    per-kernel-group figures add the implementation bytes each group moves (pooled keys,
+    centroids, the score array written by S4 and read by S5-S6)."""
+    BH, rows = w.B * w.H, w.B * w.H * w.nqb
+    qk_bytes = 2 * BH * w.N * w.d * 2
+    plan_bytes = float(counts.sum()) * 8 + rows * (4 + 16)
+    score_bytes = rows * w.nkb * 4
+    kbar_bytes = 2 * BH * w.nkb * w.d * 2       # fp16 hi + lo
+    mu_bytes = rows * 8 * w.d * (4 + 2 + 2) + rows * 8 * 4 + rows * 128
+    t = kmeans_ms + score_ms + sample_ms
+    algo = qk_bytes + plan_bytes
+
+    def gbs(nbytes, ms):
+        return nbytes / (ms * 1e-3) / 1e9
+
+    return {"bound": "hbm", "kernels": "K2 pool+k-means, K3 score (3 launches), K4 sample",
+            "algorithmic_bytes": algo, "achieved": gbs(algo, t), "peak": hbm_gbs,
+            "unit": "GB/s", "frac": gbs(algo, t) / hbm_gbs,
+            "peak_source": f"{peak_src} HBM copy bandwidth", "ms": t,
+            "per_kernel": {
+                "pool_kmeans": {"ms": kmeans_ms, "bytes": qk_bytes + kbar_bytes + mu_bytes,
+                                "gbs": gbs(qk_bytes + kbar_bytes + mu_bytes, kmeans_ms)},
+                "score": {"ms": score_ms, "bytes": score_bytes,
+                          "gbs": gbs(score_bytes, score_ms),
+                          "note": "writes the score array; reads pooled keys and centroids "
+                                  "(L2-resident); tensor + MUFU bound"},
+                "sample": {"ms": sample_ms, "bytes": score_bytes + plan_bytes,
+                           "gbs": gbs(score_bytes + plan_bytes, sample_ms)}}}
+
+
 def max_over_ranks(value, device, world):
     """The largest `value` over the ranks: a collective that every rank calls
     (with world == 1 it returns the value)."""
@@ -291,18 +355,24 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # one step: S2+S3 (pool + k-means), S4 (score), S5+S6 (sample), S7 (attention); the
+    # first two are the two halves of absa_select_scores, called separately so that each
+    # kernel group gets its own events
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        absa.select_scores(p, q, k, scores, ws)
+        absa.pool_kmeans(p, q, k, ws)
         if ev is not None:
             ev[1].record(stream)
-        absa.sample_plan(p, scores, plan)
+        absa.block_scores(p, ws, scores)
         if ev is not None:
             ev[2].record(stream)
-        absa.sparse_attention(p, q, k, v, plan, o)
+        absa.sample_plan(p, scores, plan)
         if ev is not None:
             ev[3].record(stream)
+        absa.sparse_attention(p, q, k, v, plan, o)
+        if ev is not None:
+            ev[4].record(stream)
 
     clocks = ClockSampler(dev.index).__enter__()  # sampling starts before the warm-up
     for _ in range(max(3, args.warmup)):
@@ -310,10 +380,10 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
     plan.check()
+    absa.select_check(p, ws)
 
     K = args.steps
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    attn_flops = []
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -325,16 +395,16 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     plan.check()
+    absa.select_check(p, ws)
     counts = plan.counts.to(torch.int64).cpu().numpy()
     nvalid = np.full(w.nqb, 128, np.int64)
     nvalid[-1] = w.last_valid
     # algorithmic flops of the sparse attention: 4 d per (query row, key token)
-    flops = float(4 * w.d * (counts * 4 * nvalid[None, None, :]).sum())
-    attn_flops = flops
-    sel = np.array([e[0].elapsed_time(e[1]) for e in events])
-    smp = np.array([e[1].elapsed_time(e[2]) for e in events])
-    att = np.array([e[2].elapsed_time(e[3]) for e in events])
-    tot = sel + smp + att
+    attn_flops = float(4 * w.d * (counts * 4 * nvalid[None, None, :]).sum())
+    parts = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events])
+    kmn, scr, smp, att = parts.T
+    sel = kmn + scr
+    tot = parts.sum(axis=1)
     t_local = float(tot.sum())
     t_max = max_over_ranks(t_local, dev, world)
     ms_per_call = per_call_ms(t_max, K, world)
@@ -383,26 +453,29 @@ def run_ours(args):
     peak_kind = "sustained" if long_loop else "burst"
     att_ms = float(att.mean())
     achieved_tf = attn_flops / (att_ms * 1e-3) / 1e12
-    sel_bytes = 2 * q.numel() * 2  # algorithmic: read q and k once
+    ss = selector_sampler_roofline(w, counts, float(kmn.mean()), float(scr.mean()),
+                                   float(smp.mean()), hbm_gbs, peak_src)
     line = None
     if rank == 0:
         line = {
             "metric": METRIC, "value": ms_per_call, "unit": "ms", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_max / K, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_of(w, {
-                "parallelism": f"replicas{world}" if world > 1 else "single",
+            "config": config_of(w, sampling=args.sampling),
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "per_gpu_ms": t_max / K,
+            "detail": {
                 "tflops_effective": attn_flops / (float(tot.mean()) * 1e-3) / 1e12,
                 "attention_tflops": achieved_tf,
-                "breakdown_ms": {"select_scores": float(sel.mean()), "sample": float(smp.mean()),
+                "breakdown_ms": {"pool_kmeans": float(kmn.mean()), "score": float(scr.mean()),
+                                 "select_scores": float(sel.mean()), "sample": float(smp.mean()),
                                  "sparse_attention": att_ms},
                 "plan_reuse_ms_per_call": float(sel.mean() + smp.mean()) / 4 + att_ms,
                 "dense_reference_ms": float(np.median(dense_ms)) if dense_ms else None,
                 "dense_tflops": (4.0 * w.d * w.N * w.N * w.B * w.H / (np.median(dense_ms) * 1e-3)
                                  / 1e12) if dense_ms else None,
                 "mean_blocks_per_row": float(counts.mean()),
-                "selector_hbm_frac_of_measured": sel_bytes / (float(sel.mean()) * 1e-3) / 1e9 / hbm_gbs,
-            }, sampling=args.sampling),
+            },
             "roofline": {"bound": "tensor", "kernel": "absa_attention_kernel<128,sparse>",
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": achieved_tf / peak_tf,
@@ -413,6 +486,7 @@ def run_ours(args):
                              ROOT, "block_sparse_attention_selector_b200", "csrc", "attention.cu"),
                              w),
                          "algorithmic_flops_per_launch": attn_flops},
+            "roofline_selector_sampler": ss,
             "e2e": {"value": e2e_ms, "unit": "ms",
                     "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2,
                     "api": "absa_step_host", "heads_per_run": args.e2e_heads_per_run},

@@ -11,17 +11,19 @@ import math
 
 from . import _abi
 from ._abi import (AbsaError, absa_check_params, absa_dense_reference, absa_params, absa_plan,
-                   absa_plan_capacity, absa_plan_check, absa_sample_plan, absa_select_plan,
-                   absa_select_scores, absa_sparse_attention, absa_step_host,
-                   absa_workspace_bytes)
+                   absa_plan_capacity, absa_plan_check, absa_sample_plan,
+                   absa_select_block_scores, absa_select_check, absa_select_plan,
+                   absa_select_pool_kmeans, absa_select_scores, absa_sparse_attention,
+                   absa_step_host, absa_workspace_bytes)
 from .synthetic import Workload
 
 __all__ = [
     "AbsaError", "Plan", "Workload", "absa_check_params", "absa_dense_reference", "absa_params",
     "absa_plan", "absa_plan_capacity", "absa_plan_check", "absa_sample_plan", "absa_select_plan",
+    "absa_select_block_scores", "absa_select_check", "absa_select_pool_kmeans",
     "absa_select_scores", "absa_sparse_attention", "absa_step_host", "absa_workspace_bytes",
-    "dense_reference", "make_params", "sample_plan", "select_plan", "select_scores",
-    "sparse_attention", "step_host", "workspace", "version",
+    "block_scores", "dense_reference", "make_params", "pool_kmeans", "sample_plan", "select_check",
+    "select_plan", "select_scores", "sparse_attention", "step_host", "workspace", "version",
 ]
 
 
@@ -121,6 +123,31 @@ def select_scores(p, q, k, scores=None, ws=None, stream=None):
     _abi.check(absa_select_scores(p, _ptr(q), _ptr(k), _ptr(scores), _ptr(ws), ws.numel(),
                                   _stream_handle(stream)), "absa_select_scores")
     return scores, ws
+
+
+def pool_kmeans(p, q, k, ws, stream=None):
+    """First half of select_scores: pooled keys, centroids and weights into ws."""
+    _check_bf16(q, k)
+    _abi.check(absa_select_pool_kmeans(p, _ptr(q), _ptr(k), _ptr(ws), ws.numel(),
+                                       _stream_handle(stream)), "absa_select_pool_kmeans")
+    return ws
+
+
+def block_scores(p, ws, scores=None, stream=None):
+    """Second half of select_scores: the block scores from the regions pool_kmeans wrote."""
+    import torch
+
+    nqb, nkb = (p.N + 127) // 128, (p.N + 3) // 4
+    if scores is None:
+        scores = torch.empty((p.B, p.H, nqb, nkb), dtype=torch.float32, device=ws.device)
+    _abi.check(absa_select_block_scores(p, _ptr(scores), _ptr(ws), ws.numel(),
+                                        _stream_handle(stream)), "absa_select_block_scores")
+    return scores
+
+
+def select_check(p, ws, stream=None):
+    """Synchronise and raise if the last score stage on ws gave up a bounded wait."""
+    _abi.check(absa_select_check(p, _ptr(ws), _stream_handle(stream)), "absa_select_check")
 
 
 def sample_plan(p, scores, plan=None, stream=None):

@@ -27,7 +27,8 @@ EXPORTED = (
     "absa_version", "absa_status_string", "absa_check_params", "absa_plan_capacity",
     "absa_workspace_bytes", "absa_select_scores", "absa_sample_plan", "absa_select_plan",
     "absa_sparse_attention", "absa_dense_reference", "absa_plan_check",
-    "absa_select_scores_static", "absa_step_host",
+    "absa_select_scores_static", "absa_step_host", "absa_select_pool_kmeans",
+    "absa_select_block_scores", "absa_select_check", "absa_selftest_wait_timeout",
 )
 
 ABSA_STATIC_SCRATCH_BYTES = 64 << 20
@@ -103,6 +104,14 @@ def lib():
         L.absa_step_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, Q, vp, sz,
                                      ctypes.c_int32, vp, vp, vp]
         L.absa_step_host.restype = st
+        L.absa_select_pool_kmeans.argtypes = [P, vp, vp, vp, sz, vp]
+        L.absa_select_pool_kmeans.restype = st
+        L.absa_select_block_scores.argtypes = [P, vp, vp, sz, vp]
+        L.absa_select_block_scores.restype = st
+        L.absa_select_check.argtypes = [P, vp, vp]
+        L.absa_select_check.restype = st
+        L.absa_selftest_wait_timeout.argtypes = [vp, ctypes.c_int64, vp]
+        L.absa_selftest_wait_timeout.restype = st
         _lib = L
     return _lib
 
@@ -168,3 +177,20 @@ def absa_step_host(p, q_host, k_host, v_host, o_host, q, k, v, o, scores, plan, 
     return lib().absa_step_host(ctypes.byref(p), q_host, k_host, v_host, o_host, q, k, v, o,
                                 scores, ctypes.byref(plan), ws, ws_bytes, heads_per_run, stream,
                                 copy_in_stream, copy_out_stream)
+
+
+def absa_select_pool_kmeans(p, q, k, ws, ws_bytes, stream):
+    return lib().absa_select_pool_kmeans(ctypes.byref(p), q, k, ws, ws_bytes, stream)
+
+
+def absa_select_block_scores(p, scores, ws, ws_bytes, stream):
+    return lib().absa_select_block_scores(ctypes.byref(p), scores, ws, ws_bytes, stream)
+
+
+def absa_select_check(p, ws, stream):
+    """Synchronise and read the selector's status word (ws None: the built-in array)."""
+    return lib().absa_select_check(ctypes.byref(p), ws, stream)
+
+
+def absa_selftest_wait_timeout(status, limit_cycles, stream):
+    return lib().absa_selftest_wait_timeout(status, int(limit_cycles), stream)

@@ -77,11 +77,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 
 // Wait for the phase with the given parity.  Returns false (after setting the
 // timeout flag in *status and *abort) if it does not complete within about
-// kWaitLimitCycles, or if another thread of the CTA already gave up.  After a
-// short poll the thread sleeps between checks; the clock and the abort flag
-// are read once every 16 sleeps so that waiting warps take few issue slots.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
-                                          volatile int *abort) {
+// limit_cycles SM clocks, or if another thread of the CTA already gave up.
+// After a short poll the thread sleeps between checks; the clock and the
+// abort flag are read once every 16 sleeps so that waiting warps take few
+// issue slots.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, int32_t *status,
+                                                volatile int *abort, long long limit_cycles) {
     // short non-blocking poll first: most waits end within a few hundred cycles
     // and a sleeping thread wakes up late
     for (int i = 0; i < 64; ++i)
@@ -91,13 +92,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if ((i & 15u) == 0) {
             if (*abort) return false;
-            if (clock64() - t0 > kWaitLimitCycles) {
+            if (clock64() - t0 > limit_cycles) {
                 *abort = 1;
                 if (status) atomicOr(status, ABSA_DEVFLAG_TIMEOUT);
                 return false;
             }
         }
     }
+}
+
+// mbar_wait_limit with the library's limit (kWaitLimitCycles, about a second).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
+                                          volatile int *abort) {
+    return mbar_wait_limit(bar, parity, status, abort, kWaitLimitCycles);
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

@@ -33,6 +33,11 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
                           int design, int nqb, int cap, int32_t *counts, int32_t *kv_index, float *log_pi,
                           uint64_t *r_R, int32_t *status, int64_t row0, cudaStream_t stream);
 
+// Self-test of the bounded device wait: one warp waits on an mbarrier that
+// nothing arrives at, with a limit of limit_cycles SM clocks; no copy or MMA
+// is in flight.  Sets ABSA_DEVFLAG_TIMEOUT in *status when the wait gives up.
+cudaError_t launch_wait_selftest(int32_t *status, long long limit_cycles, cudaStream_t stream);
+
 // K5 (dense = false) / K6 (dense = true): attention over 128-token tiles.
 // tq: q as [B*H*N, d] bf16 with a 64 x 128 box; tk / tv: k / v with a 64 x 4
 // box (sparse: one 4-token block per box) or a 64 x 128 box (dense tiles).

@@ -2,12 +2,36 @@
 // workspace layout, tensor maps for the TMA loads, and kernel launches on the
 // caller's stream.  No allocation, no synchronisation (except absa_plan_check).
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <mutex>
 #include <vector>
 
 #include "absa_kernels.cuh"
+
+namespace absa {
+
+// One warp waits on an mbarrier that nothing arrives at (no copy or MMA in
+// flight), so the wait must give up after limit_cycles and set the flag.
+__global__ void absa_wait_selftest_kernel(int32_t *status, long long limit_cycles) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    mbar_wait_limit(&bar, 0, status, &abort_flag, limit_cycles);
+}
+
+cudaError_t launch_wait_selftest(int32_t *status, long long limit_cycles, cudaStream_t stream) {
+    absa_wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_cycles);
+    return cudaGetLastError();
+}
+
+}  // namespace absa
 
 using namespace absa;
 
@@ -29,7 +53,7 @@ Dims dims_of(const absa_params *p) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-    size_t kbar_hi, kbar_lo, mu, mu_hi, mu_lo, w, assign, part_m, part_s, lse, total;
+    size_t kbar_hi, kbar_lo, mu, mu_hi, mu_lo, w, assign, part_m, part_s, lse, status, total;
 };
 
 WsLayout ws_layout(const absa_params *p) {
@@ -53,6 +77,7 @@ WsLayout ws_layout(const absa_params *p) {
     L.part_m = take(parts);
     L.part_s = take(parts);
     L.lse = take((size_t)dm.BH * dm.nqb * 8 * 4);
+    L.status = take(sizeof(int32_t));
     L.total = off;
     return L;
 }
@@ -103,6 +128,13 @@ bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int cols,
 bool make_map_f16(CUtensorMap *map, const void *base, int64_t rows, int cols) {
     return make_map_16(map, base, rows, cols, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
 }
+
+// An NVTX range around one entry point (visible in Nsight timelines; costs a
+// few nanoseconds when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 absa_status check_plan(const absa_params *p, const absa_plan *plan) {
     if (!plan) return ABSA_ERR_INVALID_ARG;
@@ -192,42 +224,70 @@ struct HeadRun {
 
 HeadRun all_heads(const absa_params *p) { return HeadRun{0, (int64_t)p->B * p->H}; }
 
-// Stages without argument checks (the callers check once).
-absa_status select_scores_run(const absa_params *p, const void *q, const void *k, float *scores,
-                              void *ws, int32_t *status, HeadRun hr, cudaStream_t s) {
+// Workspace regions of a run of heads.
+struct SelectPtrs {
+    __half *kb_hi, *kb_lo, *mu_hi, *mu_lo;
+    float *mu, *w, *part_m, *part_s, *lse;
+    uint8_t *assign;
+};
+
+SelectPtrs select_ptrs(const absa_params *p, void *ws, HeadRun hr) {
     const WsLayout L = ws_layout(p);
     const Dims dm = dims_of(p);
     const int64_t d = p->d;
     uint8_t *w8 = static_cast<uint8_t *>(ws);
-    auto *kb_hi = reinterpret_cast<__half *>(w8 + L.kbar_hi) + hr.bh0 * dm.nkb * d;
-    auto *kb_lo = reinterpret_cast<__half *>(w8 + L.kbar_lo) + hr.bh0 * dm.nkb * d;
-    auto *mu = reinterpret_cast<float *>(w8 + L.mu) + hr.bh0 * dm.nqb * 8 * d;
-    auto *mu_hi = reinterpret_cast<__half *>(w8 + L.mu_hi) + hr.bh0 * dm.nqb * 8 * d;
-    auto *mu_lo = reinterpret_cast<__half *>(w8 + L.mu_lo) + hr.bh0 * dm.nqb * 8 * d;
-    auto *w = reinterpret_cast<float *>(w8 + L.w) + hr.bh0 * dm.nqb * 8;
-    auto *assign = w8 + L.assign + hr.bh0 * dm.nqb * 128;
+    SelectPtrs P;
+    P.kb_hi = reinterpret_cast<__half *>(w8 + L.kbar_hi) + hr.bh0 * dm.nkb * d;
+    P.kb_lo = reinterpret_cast<__half *>(w8 + L.kbar_lo) + hr.bh0 * dm.nkb * d;
+    P.mu = reinterpret_cast<float *>(w8 + L.mu) + hr.bh0 * dm.nqb * 8 * d;
+    P.mu_hi = reinterpret_cast<__half *>(w8 + L.mu_hi) + hr.bh0 * dm.nqb * 8 * d;
+    P.mu_lo = reinterpret_cast<__half *>(w8 + L.mu_lo) + hr.bh0 * dm.nqb * 8 * d;
+    P.w = reinterpret_cast<float *>(w8 + L.w) + hr.bh0 * dm.nqb * 8;
+    P.assign = w8 + L.assign + hr.bh0 * dm.nqb * 128;
     const int64_t nkr = score_key_ranges(dm.nkb);
-    auto *part_m = reinterpret_cast<float *>(w8 + L.part_m) + hr.bh0 * nkr * dm.nqb * 8;
-    auto *part_s = reinterpret_cast<float *>(w8 + L.part_s) + hr.bh0 * nkr * dm.nqb * 8;
-    auto *lse = reinterpret_cast<float *>(w8 + L.lse) + hr.bh0 * dm.nqb * 8;
+    P.part_m = reinterpret_cast<float *>(w8 + L.part_m) + hr.bh0 * nkr * dm.nqb * 8;
+    P.part_s = reinterpret_cast<float *>(w8 + L.part_s) + hr.bh0 * nkr * dm.nqb * 8;
+    P.lse = reinterpret_cast<float *>(w8 + L.lse) + hr.bh0 * dm.nqb * 8;
+    return P;
+}
+
+int32_t *ws_status_word(const absa_params *p, void *ws) {
+    return reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + ws_layout(p).status);
+}
+
+// Stages without argument checks (the callers check once).
+// S2 + S3: pooled keys, centroids, weights and assignments into the workspace.
+absa_status pool_kmeans_run(const absa_params *p, const void *q, const void *k, void *ws,
+                            HeadRun hr, cudaStream_t s) {
+    const Dims dm = dims_of(p);
+    const int64_t d = p->d;
+    const SelectPtrs P = select_ptrs(p, ws, hr);
     const auto *qh = static_cast<const __nv_bfloat16 *>(q) + hr.bh0 * p->N * d;
     const auto *kh = static_cast<const __nv_bfloat16 *>(k) + hr.bh0 * p->N * d;
+    return from_cuda(launch_kmeans_pool(qh, kh, hr.nbh, p->N, dm.nqb, dm.nkb, p->d,
+                                        p->kmeans_iters, P.mu, P.mu_hi, P.mu_lo, P.w, P.assign,
+                                        P.kb_hi, P.kb_lo, s));
+}
+
+// S4: scores from the workspace written by pool_kmeans_run.
+absa_status block_scores_run(const absa_params *p, float *scores, void *ws, int32_t *status,
+                             HeadRun hr, cudaStream_t s) {
+    const Dims dm = dims_of(p);
+    const SelectPtrs P = select_ptrs(p, ws, hr);
     float *sh = scores + hr.bh0 * dm.nqb * (int64_t)dm.nkb;
-
     CUtensorMap tm_kb_hi, tm_kb_lo, tm_mu_hi;
-    if (!make_map_f16(&tm_kb_hi, kb_hi, hr.nbh * dm.nkb, p->d) ||
-        !make_map_f16(&tm_kb_lo, kb_lo, hr.nbh * dm.nkb, p->d) ||
-        !make_map_f16(&tm_mu_hi, mu_hi, hr.nbh * dm.nqb * 8, p->d))
+    if (!make_map_f16(&tm_kb_hi, P.kb_hi, hr.nbh * dm.nkb, p->d) ||
+        !make_map_f16(&tm_kb_lo, P.kb_lo, hr.nbh * dm.nkb, p->d) ||
+        !make_map_f16(&tm_mu_hi, P.mu_hi, hr.nbh * dm.nqb * 8, p->d))
         return ABSA_ERR_CUDA;
+    return from_cuda(launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, P.w, P.part_m, P.part_s, P.lse,
+                                  sh, hr.nbh, dm.nqb, dm.nkb, p->d, p->softmax_scale, status, s));
+}
 
-    cudaError_t e = launch_kmeans_pool(qh, kh, hr.nbh, p->N, dm.nqb, dm.nkb, p->d,
-                                       p->kmeans_iters, mu, mu_hi, mu_lo, w, assign, kb_hi, kb_lo,
-                                       s);
-    if (e != cudaSuccess) return from_cuda(e);
-    e = launch_score(tm_kb_hi, tm_kb_lo, tm_mu_hi, w, part_m, part_s, lse, sh, hr.nbh, dm.nqb,
-                     dm.nkb, p->d,
-                     p->softmax_scale, status, s);
-    return from_cuda(e);
+absa_status select_scores_run(const absa_params *p, const void *q, const void *k, float *scores,
+                              void *ws, int32_t *status, HeadRun hr, cudaStream_t s) {
+    absa_status st = pool_kmeans_run(p, q, k, ws, hr, s);
+    return st == ABSA_OK ? block_scores_run(p, scores, ws, status, hr, s) : st;
 }
 
 absa_status sample_plan_run(const absa_params *p, const float *scores, const absa_plan *plan,
@@ -270,16 +330,25 @@ absa_status attention_run(const absa_params *p, const void *q, const void *k, co
                                       plan->capacity, plan->status, s));
 }
 
+absa_status check_select_ws(const absa_params *p, const void *ws, size_t ws_bytes) {
+    if (!ws || !aligned16(ws)) return ABSA_ERR_INVALID_ARG;
+    return ws_bytes < ws_layout(p).total ? ABSA_ERR_WORKSPACE : ABSA_OK;
+}
+
+// status == nullptr: report into the workspace's status word (reset first).
 absa_status select_scores_impl(const absa_params *p, const void *q, const void *k, float *scores,
                                void *ws, size_t ws_bytes, int32_t *status, void *stream) {
     absa_status st = absa_check_params(p);
     if (st != ABSA_OK) return st;
-    if (!q || !k || !scores || !ws) return ABSA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || !aligned16(ws))
-        return ABSA_ERR_INVALID_ARG;
-    if (ws_bytes < ws_layout(p).total) return ABSA_ERR_WORKSPACE;
-    return select_scores_run(p, q, k, scores, ws, status, all_heads(p),
-                             reinterpret_cast<cudaStream_t>(stream));
+    if (!q || !k || !scores) return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return ABSA_ERR_INVALID_ARG;
+    if ((st = check_select_ws(p, ws, ws_bytes)) != ABSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!status) {
+        status = ws_status_word(p, ws);
+        if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return ABSA_ERR_CUDA;
+    }
+    return select_scores_run(p, q, k, scores, ws, status, all_heads(p), s);
 }
 
 absa_status sample_plan_impl(const absa_params *p, const float *scores, const absa_plan *plan,
@@ -326,6 +395,7 @@ extern "C" {
 
 absa_status absa_select_scores_static(const absa_params *p, const void *q, const void *k,
                                       float *scores, void *stream) {
+    NvtxRange range("absa_select_scores_static");
     absa_status st = absa_check_params(p);
     if (st != ABSA_OK) return st;
     if (ws_layout(p).total > ABSA_STATIC_SCRATCH_BYTES) return ABSA_ERR_WORKSPACE;
@@ -336,16 +406,70 @@ absa_status absa_select_scores_static(const absa_params *p, const void *q, const
 
 absa_status absa_select_scores(const absa_params *p, const void *q, const void *k, float *scores,
                                void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("absa_select_scores");
     return select_scores_impl(p, q, k, scores, ws, ws_bytes, nullptr, stream);
+}
+
+absa_status absa_select_pool_kmeans(const absa_params *p, const void *q, const void *k, void *ws,
+                                    size_t ws_bytes, void *stream) {
+    NvtxRange range("absa_select_pool_kmeans");
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (!q || !k || !aligned16(q) || !aligned16(k)) return ABSA_ERR_INVALID_ARG;
+    if ((st = check_select_ws(p, ws, ws_bytes)) != ABSA_OK) return st;
+    return pool_kmeans_run(p, q, k, ws, all_heads(p), reinterpret_cast<cudaStream_t>(stream));
+}
+
+absa_status absa_select_block_scores(const absa_params *p, float *scores, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    NvtxRange range("absa_select_block_scores");
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (!scores || !aligned16(scores)) return ABSA_ERR_INVALID_ARG;
+    if ((st = check_select_ws(p, ws, ws_bytes)) != ABSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int32_t *status = ws_status_word(p, ws);
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return ABSA_ERR_CUDA;
+    return block_scores_run(p, scores, ws, status, all_heads(p), s);
+}
+
+absa_status absa_select_check(const absa_params *p, const void *ws, void *stream) {
+    NvtxRange range("absa_select_check");
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    if (!ws) {  // the built-in array of absa_select_scores_static
+        if (ws_layout(p).total > ABSA_STATIC_SCRATCH_BYTES) return ABSA_ERR_WORKSPACE;
+        ws = static_scratch();
+        if (!ws) return ABSA_ERR_CUDA;
+    } else if (!aligned16(ws)) {
+        return ABSA_ERR_INVALID_ARG;
+    }
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ABSA_ERR_CUDA;
+    int32_t flags = 0;
+    if (cudaMemcpy(&flags, ws_status_word(p, const_cast<void *>(ws)), sizeof(flags),
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return ABSA_ERR_CUDA;
+    return (flags & ABSA_DEVFLAG_TIMEOUT) ? ABSA_ERR_TIMEOUT : ABSA_OK;
+}
+
+absa_status absa_selftest_wait_timeout(int32_t *status, int64_t limit_cycles, void *stream) {
+    NvtxRange range("absa_selftest_wait_timeout");
+    if (!status || (reinterpret_cast<uintptr_t>(status) & 3u)) return ABSA_ERR_INVALID_ARG;
+    if (limit_cycles < 1 || limit_cycles > kWaitLimitCycles) return ABSA_ERR_INVALID_ARG;
+    return from_cuda(
+        launch_wait_selftest(status, limit_cycles, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 absa_status absa_sample_plan(const absa_params *p, const float *scores, const absa_plan *plan,
                              void *stream) {
+    NvtxRange range("absa_sample_plan");
     return sample_plan_impl(p, scores, plan, true, stream);
 }
 
 absa_status absa_select_plan(const absa_params *p, const void *q, const void *k, float *scores,
                              const absa_plan *plan, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("absa_select_plan");
     absa_status st = absa_check_params(p);
     if (st != ABSA_OK) return st;
     st = check_plan(p, plan);
@@ -360,6 +484,7 @@ absa_status absa_select_plan(const absa_params *p, const void *q, const void *k,
 
 absa_status absa_sparse_attention(const absa_params *p, const void *q, const void *k,
                                   const void *v, const absa_plan *plan, void *o, void *stream) {
+    NvtxRange range("absa_sparse_attention");
     absa_status st = absa_check_params(p);
     if (st != ABSA_OK) return st;
     st = check_plan(p, plan);
@@ -373,6 +498,7 @@ absa_status absa_sparse_attention(const absa_params *p, const void *q, const voi
 
 absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,
                                  const void *v, void *o, int32_t *status, void *stream) {
+    NvtxRange range("absa_dense_reference");
     absa_status st = absa_check_params(p);
     if (st != ABSA_OK) return st;
     if (!q || !k || !v || !o) return ABSA_ERR_INVALID_ARG;
@@ -388,6 +514,7 @@ absa_status absa_step_host(const absa_params *p, const void *q_host, const void 
                            float *scores, const absa_plan *plan, void *ws, size_t ws_bytes,
                            int32_t heads_per_run, void *stream, void *copy_in_stream,
                            void *copy_out_stream) {
+    NvtxRange range("absa_step_host");
     absa_status st = absa_check_params(p);
     if (st != ABSA_OK) return st;
     st = check_plan(p, plan);
@@ -457,6 +584,7 @@ absa_status absa_step_host(const absa_params *p, const void *q_host, const void 
 }
 
 absa_status absa_plan_check(const absa_plan *plan, void *stream) {
+    NvtxRange range("absa_plan_check");
     if (!plan || !plan->status) return ABSA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(s);

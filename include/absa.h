@@ -20,8 +20,9 @@
  *    (NQB = ceil(N/128)); key/value block j holds tokens 4j .. min(4j+3, N-1)
  *    (NKB = ceil(N/4)).
  *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  The
- *    library never allocates, frees or synchronises, except absa_plan_check,
- *    which synchronises the stream to read the device status word.
+ *    library never allocates, frees or synchronises, except absa_plan_check
+ *    and absa_select_check, which synchronise the stream to read a device
+ *    status word.  Every entry point opens an NVTX range of its own name.
  *  - Pointers must be 16-byte aligned.  Host-detectable errors return before
  *    any launch; launch failures return ABSA_ERR_CUDA; errors seen on the
  *    device are OR-ed into a device status word (ABSA_DEVFLAG_*).
@@ -118,6 +119,9 @@ int32_t absa_plan_capacity(const absa_params *p);
  *                               logit minus that largest one (base 2)
  *   lse      f32  [B,H,NQB*8]   L = log2-sum-exp of the scaled logits over
  *                               all key blocks minus log2(w) (+inf if w = 0)
+ *   status   i32  [1]           device status word of the score stage
+ *                               (ABSA_DEVFLAG_TIMEOUT); read it with
+ *                               absa_select_check
  * The regions after kbar_lo are readable audit outputs of the last call.
  * Returns 0 if p is invalid. */
 size_t absa_workspace_bytes(const absa_params *p);
@@ -133,9 +137,38 @@ size_t absa_workspace_bytes(const absa_params *p);
  * on the tensor cores as fp16(mu_c) . (kbar_hi + kbar_lo); inputs whose
  * magnitude exceeds the fp16 range (65504) are clamped to it, which only
  * the accuracy of the scores can notice.  ws must hold
- * absa_workspace_bytes(p) bytes (ABSA_ERR_WORKSPACE otherwise). */
+ * absa_workspace_bytes(p) bytes (ABSA_ERR_WORKSPACE otherwise).  The call
+ * resets the workspace's status word first; a bounded wait of the score
+ * kernels that runs out sets ABSA_DEVFLAG_TIMEOUT there (the scores are then
+ * incomplete), which absa_select_check reports.  Equivalent to
+ * absa_select_pool_kmeans followed by absa_select_block_scores on the same
+ * workspace. */
 absa_status absa_select_scores(const absa_params *p, const void *q, const void *k,
                                float *scores, void *ws, size_t ws_bytes, void *stream);
+
+/* First half of absa_select_scores (IBCS paragraph: "averaged keys" and the
+ * per-block k-means): writes the kbar_hi/kbar_lo, mu, mu_hi, mu_lo, w and
+ * assign regions of ws.  The k-means kernel has no device waits and does not
+ * touch the status word.  Arguments and errors as absa_select_scores. */
+absa_status absa_select_pool_kmeans(const absa_params *p, const void *q, const void *k, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/* Second half of absa_select_scores (IBCS paragraph: weighted centroid
+ * attention to the averaged keys): the scores from the regions written by
+ * absa_select_pool_kmeans on the same ws (and the same p).  Resets the
+ * workspace's status word first.  Arguments and errors as
+ * absa_select_scores. */
+absa_status absa_select_block_scores(const absa_params *p, float *scores, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/* Synchronise `stream` and read the selector's status word: the one in ws
+ * (the workspace of absa_select_scores / absa_select_block_scores), or, with
+ * ws = NULL, the one in the built-in array of absa_select_scores_static on
+ * the current device.  Returns ABSA_ERR_TIMEOUT if the last score stage gave
+ * up a bounded wait, else ABSA_OK (also INVALID_ARG / WORKSPACE / CUDA for
+ * bad arguments or a failing CUDA call).  Does not clear the word.
+ * (absa_select_plan and absa_step_host report into plan->status instead.) */
+absa_status absa_select_check(const absa_params *p, const void *ws, void *stream);
 
 /* SIP sampler (SIP paragraph) on a score array [B,H,NQB,NKB] f32.
  * Integer inclusion probabilities: q_j = max(1, floor(s_j * 2^32)) (NaN or
@@ -211,7 +244,11 @@ absa_status absa_dense_reference(const absa_params *p, const void *q, const void
  *  - The array exists once per GPU for as long as the library is loaded in
  *    the process; the first call on a device looks up its device address
  *    (with that device current), so make that first call before any stream
- *    capture.
+ *    capture.  The address is kept for the life of the process: after
+ *    cudaDeviceReset on a device it is stale, and this entry point must not
+ *    be called on that device again.
+ *  - The array ends with the same status word as a caller workspace (reset
+ *    by every call); absa_select_check(p, NULL, stream) reads it.
  *  - Every call on a device shares the same array and leaves its contents
  *    behind; nothing in it has to start at zero (each call writes every
  *    region before reading it).  Calls that can run at the same time on one
@@ -251,6 +288,15 @@ absa_status absa_step_host(const absa_params *p, const void *q_host, const void 
                            float *scores, const absa_plan *plan, void *ws, size_t ws_bytes,
                            int32_t heads_per_run, void *stream, void *copy_in_stream,
                            void *copy_out_stream);
+
+/* Self-test of the library's bounded device waits (no counterpart on the
+ * pages; it exists so that the timeout path can be exercised without any
+ * fault): launches one warp that waits on a shared-memory barrier nothing
+ * ever completes, with no copy or MMA in flight, gives up after about
+ * limit_cycles SM clocks (1 .. 2e9) and ORs ABSA_DEVFLAG_TIMEOUT into the
+ * device word *status.  The kernel then returns normally and the context
+ * stays usable. */
+absa_status absa_selftest_wait_timeout(int32_t *status, int64_t limit_cycles, void *stream);
 
 /* Synchronise `stream`, read plan->status and map it to a status code
  * (TIMEOUT > BAD_PLAN > OVERFLOW > OK).  Does not clear the word. */

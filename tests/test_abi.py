@@ -61,9 +61,9 @@ def test_workspace_bytes_covers_layout(L):
     BH = w.B * w.H
     nkr = (w.nkb + 255) // 256
     need = (2 * BH * w.nkb * w.d * 2 + BH * w.nqb * 8 * w.d * (4 + 2 + 2) + BH * w.nqb * 8 * 4
-            + BH * w.nqb * 128 + 2 * BH * nkr * w.nqb * 8 * 4 + BH * w.nqb * 8 * 4)
+            + BH * w.nqb * 128 + 2 * BH * nkr * w.nqb * 8 * 4 + BH * w.nqb * 8 * 4 + 4)
     got = _abi.absa_workspace_bytes(p)
-    assert need <= got <= need + 10 * 256
+    assert need <= got <= need + 11 * 256
 
 
 @pytest.mark.parametrize("field,value,code", [
@@ -118,6 +118,17 @@ def test_entry_points_reject_null_and_misaligned_pointers_before_cuda(L):
                 None) == _abi.ABSA_ERR_WORKSPACE
     assert step(p, 16, 16, 16, 16, 16, 16, 16, 16, 16, bad, 16, ws, 4, None, None,
                 None) == _abi.ABSA_ERR_INVALID_ARG
+    # the two selector stages, the selector check and the wait self-test
+    assert _abi.absa_select_pool_kmeans(p, None, 16, 16, ws, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert _abi.absa_select_pool_kmeans(p, 16, 16, 8, ws, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert _abi.absa_select_pool_kmeans(p, 16, 16, 16, ws - 1, None) == _abi.ABSA_ERR_WORKSPACE
+    assert _abi.absa_select_block_scores(p, None, 16, ws, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert _abi.absa_select_block_scores(p, 16, 16, ws - 1, None) == _abi.ABSA_ERR_WORKSPACE
+    assert _abi.absa_select_check(p, 8, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert _abi.absa_select_check(_p(synthetic.WAN480), None, None) == _abi.ABSA_ERR_WORKSPACE
+    assert _abi.absa_selftest_wait_timeout(None, 1000, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert _abi.absa_selftest_wait_timeout(16, 0, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert _abi.absa_selftest_wait_timeout(16, 2_000_000_001, None) == _abi.ABSA_ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -96,3 +96,12 @@ def test_reference_arm_line_on_rank_zero():
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    # the line states what ran: ms_per_step is the measured sampled step, value the
+    # full-layer estimate from it, with the sampled query blocks and the factor
+    sw = line["sampled_work"]
+    assert line["config"]["workload"] == "hunyuan_720p_33x45x80"
+    assert 1 <= sw["timed_query_blocks_per_head"] <= sw["query_blocks_per_head"]
+    assert sw["extrapolation_factor"] == pytest.approx(
+        sw["query_blocks_per_head"] / sw["timed_query_blocks_per_head"])
+    assert line["ms_per_step"] == pytest.approx(sw["step_seconds"] * 1e3)
+    assert line["ms_per_step"] <= line["value"]
