@@ -25,13 +25,6 @@ __device__ __forceinline__ uint32_t quantise_m1(float s) {
     return __float2uint_rz(x) - 1u;     // floor for 1 <= x < 2^32
 }
 
-// Threshold t - 1 of "q >= t" on q - 1 as a u32, or `never` when t - 1 exceeds
-// every q - 1 (q <= 2^32).
-__device__ __forceinline__ uint32_t q_threshold_m1(uint64_t t, bool &never) {
-    never = t - 1 > 0xFFFFFFFFull;
-    return never ? 0xFFFFFFFFu : (uint32_t)(t - 1);
-}
-
 constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;  // SplitMix64 increment
 
 // Upper 32 bits of the SplitMix64 output function of z.  Only the high word
@@ -46,9 +39,6 @@ __device__ __forceinline__ uint32_t splitmix64_hi32(uint64_t z) {
     const uint32_t h = __umulhi(lo, 0x133111EBu) + lo * 0x94D049BBu + hi * 0x133111EBu;
     return h ^ (h >> 31);
 }
-
-// Candidate list for the capping rounds after the first (see the kernel).
-constexpr int kCandMax = 2048;
 
 // u * R < rq * 2^32 exactly (u < 2^32, R < 2^48, rq < 2^48): with
 // R = Rh 2^32 + Rl, u R = (u Rh + hi32(u Rl)) 2^32 + lo32(u Rl), so the
@@ -90,42 +80,86 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
     }
 }
 
+// Shared-memory lists of a plan row.
+constexpr int kSampleCand = 2048;  // q - 1 of the blocks at or above the list threshold
+constexpr int kSampleList = 4096;  // q - 1 of the first written entries (for the ln(pi) pass)
+
+// Scores of a row as 16-byte chunks: chunk c holds blocks 4c - off .. 4c - off + 3,
+// where off (0..3) aligns the row start to 16 bytes; blocks outside [0, nkb)
+// read as 0 and are masked by the callers.  Only the first and the last chunk
+// of a row can be partial; they are read element by element, so no load
+// leaves the row.
+struct ScoreRow {
+    const float *s;
+    const float4 *s4;
+    int nkb, off, nchunks;
+
+    __device__ ScoreRow(const float *row, int nkb_) : s(row), nkb(nkb_) {
+        off = (int)((reinterpret_cast<uintptr_t>(row) >> 2) & 3u);
+        s4 = reinterpret_cast<const float4 *>(row - off);
+        nchunks = (nkb + off + 3) >> 2;
+    }
+    __device__ float4 chunk(int c) const {
+        const int j0 = 4 * c - off;
+        if (c >= nchunks) return make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 >= 0 && j0 + 4 <= nkb) return __ldg(s4 + c);
+        float4 v;
+        v.x = (j0 >= 0 && j0 < nkb) ? __ldg(s + j0) : 0.f;
+        v.y = (j0 + 1 >= 0 && j0 + 1 < nkb) ? __ldg(s + j0 + 1) : 0.f;
+        v.z = (j0 + 2 >= 0 && j0 + 2 < nkb) ? __ldg(s + j0 + 2) : 0.f;
+        v.w = (j0 + 3 >= 0 && j0 + 3 < nkb) ? __ldg(s + j0 + 3) : 0.f;
+        return v;
+    }
+    // bit i set iff block 4c - off + i lies in [0, nkb)
+    __device__ uint32_t valid_mask(int c) const {
+        const int j0 = 4 * c - off;
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m |= (j0 + i >= 0 && j0 + i < nkb) ? 1u << i : 0u;
+        return m;
+    }
+};
+
+__device__ __forceinline__ float f4_get(const float4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
 // One CTA per plan row (b,h,qb); the grid covers rows row0 .. row0+gridDim-1
-// of the whole problem (scores and plan pointers start at row0, the hash
-// counter uses the global row).  Key blocks are handled in groups of 32 (one
-// per lane); warp w owns a contiguous run of groups, so the taken blocks of
-// warp w all precede those of warp w+1 and one scan of the 8 warp counts
-// places every entry.  Shared memory: q_j - 1 as u32 per block, one capped
-// word and one taken word (ballots) per group, and the candidate list.
-//
-// Capping: the first round (r = n, R = sum q) runs over every block and also
-// lists the blocks with 2 n q_j >= R_total, i.e. q_j at least half of the
-// first threshold R/r.  The threshold only decreases from round to round, and
-// while it stays at or above that half every block a later round caps is on
-// the list, so warp 0 runs those rounds over the list alone.  If the list
-// overflows or the threshold falls below the half, the remaining rounds scan
-// every block.  Either way the rounds are exactly those of the definition.
+// of the whole problem (scores and plan pointers start at row0, the draw
+// counter uses the global row).  The row is walked in tiles of 4 * threads
+// consecutive key blocks (thread t: the 4 blocks of chunk tile*threads + t),
+// three times:
+//  A  (from memory) q_j - 1 = quantised score, R0 = sum_j q_j, and the list of
+//     q_j at or above t_list = ceil(2^30 / n) (for scores summing to about 1 that
+//     is a quarter of the first capping threshold R0 / n, a few hundred blocks
+//     on the workloads).
+//  -  Capping rounds of the definition: C_{t+1} = {j : r_t q_j >= R_t} with
+//     r_t = n - |C_t|, R_t = R0 - sum_{C_t} q_j, from C_0 = {} until |C| stops
+//     growing.  Every capped set contains the previous one, so each round is a
+//     plain count and sum over the blocks that pass; a round runs on the list
+//     whenever its threshold R_t / r_t is at least t_list (all passing blocks
+//     are then listed), and otherwise (or if the list overflowed) over the
+//     whole row from memory.  At the fixed point, j is capped iff
+//     r* q_j >= R*.
+//  C  (from memory again; the row is still in L2) the draws and an ascending
+//     compaction: per tile, a CTA-wide scan of the per-thread taken counts
+//     places every taken block; its q - 1 goes to a shared list for the last
+//     pass.
+//  -  ln(pi) of the written entries, all threads busy (the double-precision
+//     logarithm would otherwise run once per taken lane of every warp step).
 template <int WARPS>
-__global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 5 : WARPS == 16 ? 2 : 1) absa_sample_kernel(
+__global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
     int32_t *__restrict__ counts, int32_t *__restrict__ kv_index, float *__restrict__ log_pi,
     uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, int design, int nqb) {
-    constexpr int kSampleWarps = WARPS;
-    constexpr int kSampleThreads = 32 * WARPS;
-    extern __shared__ __align__(16) uint32_t samp_smem[];
-    const int ngroups = (nkb + 31) >> 5;
-    const int ngp = (ngroups + 7) & ~7;             // groups rounded up to whole 256-block
-                                                    // super-groups (systematic pass)
-    uint32_t *qm1 = samp_smem;                      // [ngp*32]
-    uint32_t *capw = samp_smem + ngp * 32;          // [ngp]
-    uint32_t *takew = capw + ngp;                   // [ngp]
-    uint32_t *cand = takew + ngp;                   // [kCandMax]
-    __shared__ uint64_t red_a[kSampleWarps];
-    __shared__ int red_b[kSampleWarps];
-    __shared__ int warp_cnt[kSampleWarps];
+    constexpr int kThreads = 32 * WARPS;
+    __shared__ uint32_t cand[kSampleCand];
+    __shared__ uint32_t list[kSampleList];
+    __shared__ uint64_t red_a[WARPS];
+    __shared__ int red_b[WARPS];
+    __shared__ int wcnt[2][WARPS];
+    __shared__ uint64_t wmod[2][WARPS];
     __shared__ int n_cand;
-    __shared__ uint64_t fin_R;
-    __shared__ int fin_capped, fin_full;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = blockIdx.x;
@@ -134,7 +168,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 5 : WARPS == 16 ? 2 :
     float *lp_row = log_pi + row * cap;
 
     if (n >= nkb) {  // dense budget: every block, pi = 1
-        for (int j = tid; j < nkb && j < cap; j += kSampleThreads) {
+        for (int j = tid; j < nkb && j < cap; j += kThreads) {
             idx_row[j] = j;
             lp_row[j] = 0.f;
         }
@@ -147,149 +181,93 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 5 : WARPS == 16 ? 2 :
         return;
     }
 
-    const int per_warp = (ngroups + kSampleWarps - 1) / kSampleWarps;
-    const int g0 = warp * per_warp;
-    const int g1 = min(ngroups, g0 + per_warp);
-
-    // quantise once; R = sum of all q_j
-    if (tid == 0) n_cand = 0;
-    uint64_t R = 0;
-    int dummy = 0;
-    for (int g = g0; g < g1; g += 8) {  // 8 loads in flight per lane
-        float sv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = (g + u) * 32 + lane;
-            sv[u] = (g + u < g1 && j < nkb) ? __ldg(srow + j) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = (g + u) * 32 + lane;
-            if (g + u < g1 && j < nkb) {
-                const uint32_t qm = quantise_m1(sv[u]);
-                qm1[j] = qm;
-                R += (uint64_t)qm + 1;
-            }
-        }
-    }
-    block_sum2<WARPS>(R, dummy, red_a, red_b);
-    const uint64_t R0 = R;
+    const ScoreRow sr(srow, nkb);
+    const int ntiles = (sr.nchunks + kThreads - 1) / kThreads;
     const uint64_t nn = (uint64_t)n;
+    // t_list = ceil(2^30 / n) <= 2^30, compared on q - 1
+    const uint64_t t_list = ((uint64_t)1 << 30) / nn + ((((uint64_t)1 << 30) % nn) ? 1 : 0);
+    const uint32_t t_list_m1 = (uint32_t)(t_list - 1);
 
-    // round 1 over every block (r = n), listing the candidates for later rounds:
-    // n q >= R0 <=> q >= ceil(R0 / n), and 2 n q >= R0 <=> q >= ceil(R0 / (2 n)),
-    // compared on q - 1 in 32 bits
-    const uint32_t below = (1u << lane) - 1u;
-    bool never_cap, never_cand;
-    const uint32_t t_cap = q_threshold_m1((R0 + nn - 1) / nn, never_cap);
-    const uint32_t t_cand = q_threshold_m1((R0 + 2 * nn - 1) / (2 * nn), never_cand);
-    uint64_t capsum = 0;
-    int capcnt = 0;
-    for (int g = g0; g < g1; ++g) {
-        const int j = g * 32 + lane;
-        bool newcap = false, is_cand = false;
-        if (j < nkb) {
-            const uint32_t qm = qm1[j];
-            if (!never_cap && qm >= t_cap) {
-                newcap = true;
-                capsum += (uint64_t)qm + 1;
-                ++capcnt;
-            } else if (!never_cand && qm >= t_cand) {
-                is_cand = true;
-            }
-        }
-        const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
-        if (lane == 0) capw[g] = nb;
-        const uint32_t cb = __ballot_sync(0xffffffffu, is_cand);
-        if (cb) {
-            int base = 0;
-            if (lane == 0) base = atomicAdd(&n_cand, __popc(cb));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const int p = base + __popc(cb & below);
-            if (is_cand && p < kCandMax) cand[p] = (uint32_t)j;
-        }
-    }
-    block_sum2<WARPS>(capsum, capcnt, red_a, red_b);
-    int n_capped = capcnt;
-    uint64_t r = nn - (uint64_t)n_capped;
-    R = R0 - capsum;
-
-    // later rounds over the candidate list (warp 0)
-    if (warp == 0) {
-        const int nc = n_cand;
-        bool full = nc > kCandMax;
-        bool grew = capcnt > 0;
-        while (grew && !full) {
-            // the list holds every block this round can cap iff R / r >= R0 / (2 n)
-            if ((unsigned __int128)(2 * nn) * R < (unsigned __int128)r * R0) {
-                full = true;
-                break;
-            }
-            uint64_t s = 0;
-            int c = 0;
-            for (int i = lane; i < nc; i += 32) {
-                const uint32_t j = cand[i];
-                if (!((capw[j >> 5] >> (j & 31)) & 1u)) {
-                    const uint64_t q = (uint64_t)qm1[j] + 1;
-                    if (r * q >= R) {
-                        s += q;
-                        ++c;
-                        atomicOr(&capw[j >> 5], 1u << (j & 31));
-                    }
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                s += __shfl_xor_sync(0xffffffffu, s, o);
-                c += __shfl_xor_sync(0xffffffffu, c, o);
-            }
-            grew = c > 0;
-            n_capped += c;
-            r -= (uint64_t)c;
-            R -= s;
-            __syncwarp();  // this round's marks are visible to the next round's reads
-        }
-        if (lane == 0) {
-            fin_R = R;
-            fin_capped = n_capped;
-            fin_full = full ? 1 : 0;
-        }
-    }
+    // ---- pass A: R0 and the candidate list
+    if (tid == 0) n_cand = 0;
     __syncthreads();
-    R = fin_R;
-    n_capped = fin_capped;
-    r = nn - (uint64_t)n_capped;
-    if (fin_full) {
-        // remaining rounds scan every block (the state so far is exact)
-        for (;;) {
-            uint64_t newsum = 0;
-            int grew = 0;
-            for (int g = g0; g < g1; ++g) {
-                const int j = g * 32 + lane;
-                const uint32_t word = capw[g];
-                bool newcap = false;
-                if (j < nkb && !((word >> lane) & 1u)) {
-                    const uint64_t q = (uint64_t)qm1[j] + 1;
-                    if (r * q >= R) {
-                        newcap = true;
-                        newsum += q;
+    uint64_t R0 = 0;
+    {
+        constexpr int kAhead = 4;  // tiles in flight per thread
+        for (int t0 = 0; t0 < ntiles; t0 += kAhead) {
+            float4 v[kAhead];
+#pragma unroll
+            for (int u = 0; u < kAhead; ++u) v[u] = sr.chunk((t0 + u) * kThreads + tid);
+#pragma unroll
+            for (int u = 0; u < kAhead; ++u) {
+                const int c = (t0 + u) * kThreads + tid;
+                const uint32_t valid = sr.valid_mask(c);
+                uint32_t qm[4];
+                int nc = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    qm[i] = quantise_m1(f4_get(v[u], i));
+                    if ((valid >> i) & 1u) {
+                        R0 += (uint64_t)qm[i] + 1;
+                        nc += qm[i] >= t_list_m1 ? 1 : 0;
                     }
                 }
-                const uint32_t nb = __ballot_sync(0xffffffffu, newcap);
-                if (nb) {
-                    if (lane == 0) capw[g] = word | nb;
-                    grew += lane == 0 ? __popc(nb) : 0;
+                if (nc) {  // rare: append this thread's listed blocks
+                    int p = atomicAdd(&n_cand, nc);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (((valid >> i) & 1u) && qm[i] >= t_list_m1) {
+                            if (p < kSampleCand) cand[p] = qm[i];
+                            ++p;
+                        }
                 }
             }
-            block_sum2<WARPS>(newsum, grew, red_a, red_b);
-            if (grew == 0) break;
-            n_capped += grew;
-            r = nn - (uint64_t)n_capped;
-            R -= newsum;
         }
     }
-    const uint32_t r32 = (uint32_t)r;  // r <= n < NKB < 2^16
+    int dummy = 0;
+    block_sum2<WARPS>(R0, dummy, red_a, red_b);  // its barriers also publish n_cand and cand
+    const int nc_total = n_cand;
+    const bool list_ok = nc_total <= kSampleCand;
 
+    // ---- capping rounds
+    uint64_t r = nn, R = R0;
+    int n_capped = 0;
+    for (;;) {
+        uint64_t sum = 0;
+        int c = 0;
+        if (list_ok && R >= r * t_list) {
+            for (int i = tid; i < nc_total; i += kThreads) {
+                const uint64_t q = (uint64_t)cand[i] + 1;
+                if (r * q >= R) {
+                    sum += q;
+                    ++c;
+                }
+            }
+        } else {
+            for (int t = 0; t < ntiles; ++t) {
+                const int ch = t * kThreads + tid;
+                const float4 v = sr.chunk(ch);
+                const uint32_t valid = sr.valid_mask(ch);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint64_t q = (uint64_t)quantise_m1(f4_get(v, i)) + 1;
+                    if (((valid >> i) & 1u) && r * q >= R) {
+                        sum += q;
+                        ++c;
+                    }
+                }
+            }
+        }
+        block_sum2<WARPS>(sum, c, red_a, red_b);
+        if (c == n_capped) break;  // the capped set stopped growing
+        n_capped = c;
+        r = nn - (uint64_t)c;
+        R = R0 - sum;
+    }
+    const uint32_t r32 = (uint32_t)r;  // 1 <= r <= n < NKB < 2^16
+    const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
+
+    // ---- pass C: draws and ascending compaction
     // SplitMix64 state of block j is base + j * gamma with
     // base = mix(seed) + (draw row * NKB + 1) * gamma; the draw row is the
     // global row, or under the paired design that of the even query block of
@@ -298,137 +276,116 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 5 : WARPS == 16 ? 2 :
     const int64_t drow =
         row0 + row - (design == ABSA_SAMPLING_PAIRED ? (int)(blockIdx.x % (unsigned)nqb) & 1 : 0);
     const uint64_t base = splitmix64_mix(seed) + ((uint64_t)drow * (uint64_t)nkb + 1) * kGamma;
-    const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
-    int taken = 0;
-    if (design != ABSA_SAMPLING_SYSTEMATIC) {
-        // Poisson draws (own or paired counters): one taken word per group
-        uint64_t state = base + (uint64_t)(g0 * 32 + lane) * kGamma;  // state of block j
-        for (int g = g0; g < g1; ++g, state += 32 * kGamma) {
-            const int j = g * 32 + lane;
-            bool take = false;
-            if (j < nkb) {
-                if ((capw[g] >> lane) & 1u) {
-                    take = true;
-                } else {
-                    const uint64_t rq = (uint64_t)r32 * qm1[j] + r32;
-                    take = draw_taken(splitmix64_hi32(state), Rh, Rl, rq);
-                }
-            }
-            const uint32_t tw = __ballot_sync(0xffffffffu, take);
-            if (lane == 0) takew[g] = tw;
-            taken += __popc(tw);
-        }
-    } else {
-        // Systematic design.  Interval j is [A_j, A_j + a_j) with a_j = R on C
-        // and r q_j elsewhere, A_j = sum_{i<j} a_i; the points are
-        // (k + U/2^32) R.  With rho_j = A_j mod R (capped blocks add 0 mod R)
-        // and F = floor(U R / 2^32), an uncapped interval (a_j < R) holds the
-        // point of its own period iff rho_j <= F < rho_j + a_j and that of
-        // the next period iff R + F < rho_j + a_j (comparisons of the exact
-        // values U R vs multiples of 2^32 reduce to these on F).
-        // Blocks go in super-groups of 256: lane l holds the 8 consecutive
-        // blocks 8l..8l+7, sums them in order and one warp scan per
-        // super-group gives each lane its starting rho; the 8 taken bits are
-        // the lane's byte of the group's taken word.
+    const bool systematic = design == ABSA_SAMPLING_SYSTEMATIC;
+    // Systematic design.  Interval j is [A_j, A_j + a_j) with a_j = R on C and
+    // r q_j elsewhere, A_j = sum_{i<j} a_i; the points are (k + U/2^32) R.
+    // With rho_j = A_j mod R (capped blocks add 0 mod R) and
+    // F = floor(U R / 2^32), an uncapped interval (a_j < R) holds the point of
+    // its own period iff rho_j <= F < rho_j + a_j and that of the next period
+    // iff R + F < rho_j + a_j (comparisons of the exact values U R vs multiples
+    // of 2^32 reduce to these on F).  rho comes from a CTA-wide scan mod R per
+    // tile, carried across tiles.
+    uint64_t F = 0;
+    if (systematic) {
         const uint32_t U = splitmix64_hi32(base);  // the draw of block 0 of the row
-        const uint64_t F = (uint64_t)U * Rh + __umulhi(U, Rl);
-        const int nsg = ngp >> 3;
-        const int sg_per_warp = (nsg + kSampleWarps - 1) / kSampleWarps;
-        const int s0 = warp * sg_per_warp, s1 = min(nsg, s0 + sg_per_warp);
-        // a_j mod R of the lane's 8 blocks (0 when capped or past NKB) and their capped bits
-        auto elems = [&](int sg, uint64_t (&e)[8], uint32_t &cb) {
-            const int j0 = sg * 256 + lane * 8;
-            const uint4 v0 = *reinterpret_cast<const uint4 *>(qm1 + j0);
-            const uint4 v1 = *reinterpret_cast<const uint4 *>(qm1 + j0 + 4);
-            const uint32_t qv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const int valid = min(8, max(0, nkb - j0));
-            cb = (capw[j0 >> 5] >> (j0 & 31)) & ((1u << valid) - 1u);
+        F = (uint64_t)U * Rh + __umulhi(U, Rl);
+    }
+    uint64_t rho_carry = 0;
+    int total = 0;
+    float4 v = sr.chunk(tid);
+    for (int t = 0; t < ntiles; ++t) {
+        const int ch = t * kThreads + tid;
+        const float4 vn = sr.chunk(ch + kThreads);  // next tile, in flight during this one
+        const uint32_t valid = sr.valid_mask(ch);
+        const int j0 = 4 * ch - sr.off;
+        uint32_t qm[4];
+        uint64_t rq[4];
+        uint32_t capped = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                e[i] = (i < valid && !((cb >> i) & 1u)) ? (uint64_t)r32 * qv[i] + r32 : 0;
-        };
-        uint64_t tot = 0;
-        for (int sg = s0; sg < s1; ++sg) {
-            uint64_t e[8];
-            uint32_t cb;
-            elems(sg, e, cb);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) tot = addmod(tot, e[i], R);
+        for (int i = 0; i < 4; ++i) {
+            qm[i] = quantise_m1(f4_get(v, i));
+            rq[i] = (uint64_t)r32 * qm[i] + r32;
+            if (((valid >> i) & 1u) && rq[i] >= R) capped |= 1u << i;
         }
+        uint32_t bits = capped;
+        if (!systematic) {
+            uint64_t state = base + (uint64_t)(int64_t)j0 * kGamma;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tot = addmod(tot, __shfl_xor_sync(0xffffffffu, tot, o), R);
-        __syncthreads();  // earlier readers of red_a are done
-        if (lane == 0) red_a[warp] = tot;
-        __syncthreads();
-        uint64_t carry = 0;  // rho of this warp's first block
-        for (int w = 0; w < warp; ++w) carry = addmod(carry, red_a[w], R);
-        uint8_t *takeb = reinterpret_cast<uint8_t *>(takew);
-        for (int sg = s0; sg < s1; ++sg) {
-            uint64_t e[8];
-            uint32_t cb;
-            elems(sg, e, cb);
-            uint64_t lt = 0;
+            for (int i = 0; i < 4; ++i, state += kGamma)
+                if (((valid & ~capped) >> i) & 1u)
+                    bits |= draw_taken(splitmix64_hi32(state), Rh, Rl, rq[i]) ? 1u << i : 0u;
+        } else {
+            uint64_t e[4], lsum = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) lt = addmod(lt, e[i], R);
-            uint64_t inc = lt;  // inclusive scan of the lane totals, mod R
+            for (int i = 0; i < 4; ++i) {
+                e[i] = (((valid & ~capped) >> i) & 1u) ? rq[i] : 0;  // a_j mod R
+                lsum = addmod(lsum, e[i], R);
+            }
+            uint64_t inc = lsum;  // inclusive warp scan mod R
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc = addmod(inc, y, R);
             }
-            uint64_t rho = addmod(carry, submod(inc, lt, R), R);
-            uint32_t bits = cb;
+            if (lane == 31) wmod[t & 1][warp] = inc;
+            __syncthreads();
+            uint64_t rho = rho_carry, tile_sum = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int w = 0; w < WARPS; ++w) {
+                const uint64_t x = wmod[t & 1][w];
+                if (w < warp) rho = addmod(rho, x, R);
+                tile_sum = addmod(tile_sum, x, R);
+            }
+            rho = addmod(rho, submod(inc, lsum, R), R);
+            rho_carry = addmod(rho_carry, tile_sum, R);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
                 const uint64_t a = e[i];
                 if (a != 0 && ((rho <= F && F < rho + a) || R + F < rho + a)) bits |= 1u << i;
                 rho = addmod(rho, a, R);
             }
-            takeb[sg * 32 + lane] = (uint8_t)bits;  // byte lane&3 of group word sg*8 + lane/4
-            carry = addmod(carry, __shfl_sync(0xffffffffu, inc, 31), R);
         }
-        __syncthreads();  // taken words written by other warps
-        for (int g = g0 + lane; g < g1; g += 32) taken += __popc(takew[g]);
+        // CTA-wide exclusive scan of the taken counts
+        const int cnt = __popc(bits);
+        int inc = cnt;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) taken += __shfl_xor_sync(0xffffffffu, taken, o);
-    }
-    if (lane == 0) warp_cnt[warp] = taken;
-    __syncthreads();
-    int pos = 0, total = 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (lane == 31) wcnt[t & 1][warp] = inc;
+        __syncthreads();
+        int pos = total, tile_total = 0;
 #pragma unroll
-    for (int w = 0; w < kSampleWarps; ++w) {
-        const int c = warp_cnt[w];
-        pos += w < warp ? c : 0;
-        total += c;
-    }
-    // ascending compaction of this warp's run (block ids only); the ids are
-    // also kept in shared memory (the candidate list is no longer needed)
-    // for the logarithm pass when they fit
-    const bool ids_in_smem = min(total, cap) <= kCandMax;
-    for (int g = g0; g < g1 && pos < cap; ++g) {
-        const uint32_t tw = takew[g];
-        if ((tw >> lane) & 1u) {
-            const int p = pos + __popc(tw & below);
-            if (p < cap) {
-                idx_row[p] = g * 32 + lane;
-                if (ids_in_smem) cand[p] = (uint32_t)(g * 32 + lane);
+        for (int w = 0; w < WARPS; ++w) {
+            const int x = wcnt[t & 1][w];
+            pos += w < warp ? x : 0;
+            tile_total += x;
+        }
+        pos += inc - cnt;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if ((bits >> i) & 1u) {
+                if (pos < cap) {
+                    idx_row[pos] = j0 + i;
+                    if (pos < kSampleList) list[pos] = qm[i];
+                }
+                ++pos;
             }
-        }
-        pos += __popc(tw);
+        total += tile_total;
+        v = vn;
     }
-    __syncthreads();  // the block ids written above are visible to the whole CTA
-    // ln(pi) of the written entries, all lanes busy (the double-precision
-    // logarithm would otherwise run for a whole warp per taken lane)
+    __syncthreads();  // list and the kv_index entries are visible to the whole CTA
+
+    // ---- ln(pi) of the written entries
     const int written = min(total, cap);
-    for (int p = tid; p < written; p += kSampleThreads) {
-        const int j = ids_in_smem ? (int)cand[p] : idx_row[p];
-        float lp = 0.f;
-        if (!((capw[j >> 5] >> (j & 31)) & 1u))
-            lp = (float)log((double)((uint64_t)r32 * qm1[j] + r32) / (double)R);
-        lp_row[p] = lp;
+    for (int p = tid; p < written; p += kThreads) {
+        const uint32_t qmp = p < kSampleList ? list[p] : quantise_m1(__ldg(srow + idx_row[p]));
+        const uint64_t rqp = (uint64_t)r32 * qmp + r32;
+        lp_row[p] = rqp >= R ? 0.f : (float)log((double)rqp / (double)R);
     }
     if (tid == 0) {
-        counts[row] = min(total, cap);
+        counts[row] = written;
         r_R[2 * row] = r;
         r_R[2 * row + 1] = R;
         if (total > cap) atomicOr(status, ABSA_DEVFLAG_OVERFLOW);
@@ -439,11 +396,8 @@ template <int WARPS>
 static cudaError_t launch_sample_w(const float *scores, int64_t rows, int nkb, int64_t n,
                                    uint64_t seed, int design, int nqb, int cap, int32_t *counts,
                                    int32_t *kv_index, float *log_pi, uint64_t *r_R,
-                                   int32_t *status, int64_t row0, int smem, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(absa_sample_kernel<WARPS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    absa_sample_kernel<WARPS><<<(unsigned)rows, 32 * WARPS, smem, stream>>>(
+                                   int32_t *status, int64_t row0, cudaStream_t stream) {
+    absa_sample_kernel<WARPS><<<(unsigned)rows, 32 * WARPS, 0, stream>>>(
         scores, nkb, n, seed, cap, counts, kv_index, log_pi, r_R, status, row0, design, nqb);
     return cudaGetLastError();
 }
@@ -452,20 +406,13 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
                           int design, int nqb, int cap, int32_t *counts, int32_t *kv_index,
                           float *log_pi, uint64_t *r_R, int32_t *status, int64_t row0,
                           cudaStream_t stream) {
-    const int ngroups = (nkb + 31) / 32;
-    const int ngp = (ngroups + 7) & ~7;
-    const int smem = (ngp * 32 + 2 * ngp + kCandMax) * 4;
-    // The shared score copy limits the CTAs per SM (228 KB, 1 KB reserved
-    // per CTA); wider CTAs keep about 32 warps per SM when few CTAs fit.
-    const int per_sm = (228 * 1024) / (smem + 1024);
-    if (per_sm >= 4)
-        return launch_sample_w<8>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
-                                  log_pi, r_R, status, row0, smem, stream);
-    if (per_sm >= 2)
+    // Wider CTAs for long rows keep fewer rows in flight, so that a row read by
+    // the first pass is still in L2 when the draw pass reads it again.
+    if (nkb >= 16384)
         return launch_sample_w<16>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
-                                   log_pi, r_R, status, row0, smem, stream);
-    return launch_sample_w<32>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
-                               log_pi, r_R, status, row0, smem, stream);
+                                   log_pi, r_R, status, row0, stream);
+    return launch_sample_w<8>(scores, rows, nkb, n, seed, design, nqb, cap, counts, kv_index,
+                              log_pi, r_R, status, row0, stream);
 }
 
 }  // namespace absa

@@ -211,3 +211,43 @@ def test_paired_full_layer_plans_nest():
             t_lo = np.where(lo0, takes[0], takes[1])
             t_hi = np.where(lo0, takes[1], takes[0])
             assert not np.any(t_lo & ~t_hi), (h, qb)
+
+
+# Rows that leave the sampler's fast path: the kernel keeps a shared list of
+# the largest quantised scores (those at or above ceil(2^30 / n)) and runs the
+# capping rounds on it while their threshold stays above the list's; rows whose
+# scores do not sum to about 1 overflow the list (sum far above 1) or start
+# below its threshold (sum far below 1), and then every round re-reads the
+# whole row.  Special values exercise the quantisation: NaN, negative and
+# zero scores count as q = 1, scores of 1 or more as q = 2^32.  The row
+# lengths 515 and 8190 put row starts off 16-byte boundaries.
+def _odd_rows(rows, nkb, seed):
+    rng = np.random.default_rng([seed, 5])
+    s = synthetic.random_scores(rows, nkb, seed, concentration=1.5).astype(np.float64)
+    scale = np.array([1.0, 1e3, 1e-3, 7.0, 1e-6, 1.0, 0.5, 2.0])[np.arange(rows) % 8]
+    s = (s * scale[:, None]).astype(np.float32)
+    special = rows // 8 * 8 - 3 if rows >= 8 else rows - 1  # one row with special values
+    idx = rng.choice(nkb, size=min(nkb, 12), replace=False)
+    s[special, idx[:3]] = np.nan
+    s[special, idx[3:6]] = -0.25
+    s[special, idx[6:8]] = 0.0
+    s[special, idx[8:10]] = 1.0
+    s[special, idx[10:]] = 3.5
+    return s
+
+
+@pytest.mark.parametrize("design", ["poisson", "systematic", "paired"])
+@pytest.mark.parametrize("nkb,H,n,seed", [(515, 3, 37, 21), (8190, 1, 819, 22),
+                                          (29700, 1, 2376, 23)])
+def test_sampler_fallback_paths_and_special_values(design, nkb, H, n, seed):
+    import torch
+
+    p = _params(nkb, H, n, seed, sampling=design)
+    nqb = (p.N + 127) // 128
+    scores = _odd_rows(H * nqb, nkb, seed).reshape(1, H, nqb, nkb)
+    plan = sample_plan(p, torch.from_numpy(scores).cuda())
+    try:
+        plan.check()
+    except AbsaError as e:  # rows far from normalised can overflow the capacity
+        assert e.code == _abi.ABSA_ERR_PLAN_OVERFLOW
+    _compare(p, scores, plan, plan.capacity)
