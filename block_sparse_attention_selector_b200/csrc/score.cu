@@ -26,7 +26,8 @@ namespace absa {
 
 constexpr int kScoreKeyTiles = 2;                    // key tiles (128 key blocks) per CTA
 constexpr int kScoreRange = 128 * kScoreKeyTiles;    // key blocks per CTA
-constexpr int kScoreThreads = 320;                   // 0 TMA, 1 MMA, 2..9 epilogue
+constexpr int kScoreGroupWarps = 8;                  // epilogue warps per group
+constexpr int kScoreThreads = 32 * (2 + 2 * kScoreGroupWarps);  // 0 TMA, 1 MMA, 2..17 epilogue
 
 template <int D>
 struct Score2Smem {
@@ -40,8 +41,8 @@ struct Score2Smem {
     static constexpr int kKeyLoOff = kRegions * kKeyRegion;      // lo parts after the hi parts
     static constexpr int kKeyOff = 0;
     static constexpr int kMuOff = kScoreKeyTiles * kKeyTileBytes;  // 2-stage centroid ring
-    static constexpr int kXOff = kMuOff + 2 * kMuTileBytes;      // f32 [2][2][128] half exchange
-    static constexpr int kBarOff = kXOff + 2 * 2 * 128 * 4;
+    static constexpr int kXOff = kMuOff + 2 * kMuTileBytes;      // f32 [group][slot][2][128] exchange
+    static constexpr int kBarOff = kXOff + 2 * 2 * 2 * 128 * 4;
     static constexpr int kBytes = kBarOff + 16 * 8;
     // one CTA per SM: every CTA holds all 512 TMEM columns
     static constexpr int kAlloc = (kBytes + 1024 > 120 * 1024) ? kBytes + 1024 : 120 * 1024;
@@ -81,7 +82,7 @@ struct ScoreCta {
                 mbar_init(mu_full + s, 1);
                 mbar_init(mu_empty + s, 1);
                 mbar_init(d_full + s, 1);
-                mbar_init(d_empty + s, 8);
+                mbar_init(d_empty + s, kScoreGroupWarps);
             }
             *abort_flag = 0;
             mbar_fence_init();
@@ -198,16 +199,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1) absa_score_lse_kernel(
     } else if (warp == 1) {
         if (lane == 0) cta.mma(tmem, nmt, status);
     } else {
-        const int quarter = warp & 3, half = (warp - 2) >> 2;
+        // epilogue group g takes the centroid tiles m = g, g + 2, ... (TMEM
+        // buffer g), so one group's exponentials overlap the other's loads,
+        // maxima and exchange; within a group, warp w: TMEM lane quarter
+        // w % 4, key tile (w % 8) / 4
+        const int e = warp - 2, g = e / kScoreGroupWarps, we = e % kScoreGroupWarps;
+        const int quarter = warp & 3, half = we >> 2;
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + half * 128;
         const int ncols = min(128, nkb - kr * kScoreRange - half * 128);  // valid key blocks
-        float *xch = reinterpret_cast<float *>(cta.sm + S::kXOff);      // [m&1][max|sum][row]
-        // every epilogue warp passes the named barrier once per centroid tile,
-        // also after a failed wait (then without touching TMEM)
+        float *xch = reinterpret_cast<float *>(cta.sm + S::kXOff);  // [g][slot][max|sum][row]
+        // every warp of a group passes the group's named barrier once per tile
+        // of the group, also after a failed wait (then without touching TMEM)
         bool ok = true;
-        for (int m = 0; m < nmt; ++m) {
-            const int buf = m & 1;
+        for (int m = g; m < nmt; m += 2) {
+            const int buf = g;
             if (ok)
                 ok = __all_sync(0xffffffffu,
                                 mbar_wait(cta.d_full + buf, (m >> 1) & 1, status, cta.abort_flag));
@@ -247,13 +253,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1) absa_score_lse_kernel(
                     a4[i & 3] += ex2(__fmaf_rn(__uint_as_float(v[i >> 5][i & 31]), scale_log2, moff));
                 sum += (a4[0] + a4[1]) + (a4[2] + a4[3]);
             }
+            // two exchange slots per group, alternating with the group's tiles:
+            // a slot is rewritten two group tiles later, after the group's
+            // barrier of the tile in between
+            float *x = xch + (g * 2 + ((m >> 1) & 1)) * 256;
             if (half == 1) {
-                xch[buf * 256 + r] = mx;
-                xch[buf * 256 + 128 + r] = sum;
+                x[r] = mx;
+                x[128 + r] = sum;
             }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            asm volatile("bar.sync %0, 256;" ::"r"(1 + g) : "memory");
             if (half == 0 && ok) {
-                const float m1 = xch[buf * 256 + r], s1 = xch[buf * 256 + 128 + r];
+                const float m1 = x[r], s1 = x[128 + r];
                 const float mm = fmaxf(mx, m1);
                 const float tot = (mx == -INFINITY ? 0.f : sum * ex2((mx - mm) * scale_log2)) +
                                   (m1 == -INFINITY ? 0.f : s1 * ex2((m1 - mm) * scale_log2));
@@ -314,58 +324,64 @@ __global__ void __launch_bounds__(kScoreThreads, 1) absa_score_out_kernel(
     } else if (warp == 1) {
         if (lane == 0) cta.mma(tmem, nmt, status);
     } else {
-        const int quarter = warp & 3, half = (warp - 2) >> 2;
+        // epilogue group g takes the centroid tiles m = g, g + 2, ... (TMEM
+        // buffer g); within a group, warp w: TMEM lane quarter w % 4 (key
+        // blocks), key tile (w % 8) / 4
+        const int e8 = warp - 2, g = e8 / kScoreGroupWarps, we = e8 % kScoreGroupWarps;
+        const int quarter = warp & 3, half = we >> 2;
         const int j = kr * kScoreRange + half * 128 + quarter * 32 + lane;  // key block
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + half * 128;
         const float *Lh = L + bh * (int64_t)nrows;
         float *sh = scores + bh * (int64_t)nqb * nkb;
-        // L of the centroid tile in shared memory (double-buffered by tile
-        // parity); epilogue thread e < 128 fetches row e of the next tile while
-        // the current one is processed
-        float *Ls = reinterpret_cast<float *>(cta.sm + Score2Smem<D>::kXOff);  // [2][128]
-        const int e = (warp - 2) * 32 + lane;
-        float lnext = (e < 128 && e < nrows) ? __ldg(Lh + e) : INFINITY;
+        // L of the group's centroid tile in shared memory (two slots per group,
+        // alternating with its tiles); group thread e < 128 fetches row e of
+        // the group's next tile while the current one is processed
+        float *Lg = reinterpret_cast<float *>(cta.sm + Score2Smem<D>::kXOff) + g * 256;
+        const int e = we * 32 + lane;
+        float lnext = (g * 128 + e < nrows && g < nmt) ? __ldg(Lh + g * 128 + e) : INFINITY;
         bool ok = true;
-        for (int m = 0; m < nmt; ++m) {
-            const int buf = m & 1;
-            if (e < 128) Ls[buf * 128 + e] = lnext;
-            asm volatile("bar.sync 1, 256;" ::: "memory");  // every epilogue warp, every tile
-            if (e < 128 && m + 1 < nmt) {
-                const int row = (m + 1) * 128 + e;
+        for (int m = g; m < nmt; m += 2) {
+            const int buf = g;
+            float *Ls = Lg + ((m >> 1) & 1) * 128;
+            if (e < 128) Ls[e] = lnext;
+            asm volatile("bar.sync %0, 256;" ::"r"(1 + g) : "memory");  // every warp, every tile
+            if (e < 128 && m + 2 < nmt) {
+                const int row = (m + 2) * 128 + e;
                 lnext = row < nrows ? __ldg(Lh + row) : INFINITY;
             }
             if (ok)
                 ok = __all_sync(0xffffffffu,
                                 mbar_wait(cta.d_full + buf, (m >> 1) & 1, status, cta.abort_flag));
-            if (!ok) continue;
-            tc_fence_after();
+            if (ok) {
+                tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {  // 64 centroid columns = 8 query blocks
-                uint32_t v[2][32];
-                tmem_ld32(lane_addr + buf * 256 + ch * 64, v[0]);
-                tmem_ld32(lane_addr + buf * 256 + ch * 64 + 32, v[1]);
-                tmem_wait_ld();
-                if (ch == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(cta.d_empty + buf);
-                }
-                if (j >= nkb) continue;
-#pragma unroll
-                for (int qbl = 0; qbl < 8; ++qbl) {
-                    const int qb = m * 16 + ch * 8 + qbl;
-                    if (qb >= nqb) break;
-                    const float4 L0 = *reinterpret_cast<const float4 *>(Ls + buf * 128 + (ch * 8 + qbl) * 8);
-                    const float4 L1 = *reinterpret_cast<const float4 *>(Ls + buf * 128 + (ch * 8 + qbl) * 8 + 4);
-                    const float Lc[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
-                    float s2[2] = {0.f, 0.f};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int col = qbl * 8 + c;
-                        s2[c & 1] += ex2(__fmaf_rn(__uint_as_float(v[col >> 5][col & 31]),
-                                                   scale_log2, -Lc[c]));
+                for (int ch = 0; ch < 2; ++ch) {  // 64 centroid columns = 8 query blocks
+                    uint32_t v[2][32];
+                    tmem_ld32(lane_addr + buf * 256 + ch * 64, v[0]);
+                    tmem_ld32(lane_addr + buf * 256 + ch * 64 + 32, v[1]);
+                    tmem_wait_ld();
+                    if (ch == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(cta.d_empty + buf);
                     }
-                    sh[(int64_t)qb * nkb + j] = s2[0] + s2[1];
+                    if (j >= nkb) continue;
+#pragma unroll
+                    for (int qbl = 0; qbl < 8; ++qbl) {
+                        const int qb = m * 16 + ch * 8 + qbl;
+                        if (qb >= nqb) break;
+                        const float4 L0 = *reinterpret_cast<const float4 *>(Ls + (ch * 8 + qbl) * 8);
+                        const float4 L1 = *reinterpret_cast<const float4 *>(Ls + (ch * 8 + qbl) * 8 + 4);
+                        const float Lc[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
+                        float s2[2] = {0.f, 0.f};
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int col = qbl * 8 + c;
+                            s2[c & 1] += ex2(__fmaf_rn(__uint_as_float(v[col >> 5][col & 31]),
+                                                       scale_log2, -Lc[c]));
+                        }
+                        sh[(int64_t)qb * nkb + j] = s2[0] + s2[1];
+                    }
                 }
             }
         }
