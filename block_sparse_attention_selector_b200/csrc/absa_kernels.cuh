@@ -38,9 +38,11 @@ cudaError_t launch_sample(const float *scores, int64_t rows, int nkb, int64_t n,
 // is in flight.  Sets ABSA_DEVFLAG_TIMEOUT in *status when the wait gives up.
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_cycles, cudaStream_t stream);
 
-// K5 (dense = false) / K6 (dense = true): attention over 128-token tiles.
-// tq: q as [B*H*N, d] bf16 with a 64 x 128 box; tk / tv: k / v with a 64 x 4
-// box (sparse: one 4-token block per box) or a 64 x 128 box (dense tiles).
+// K5 (dense = false) / K6 (dense = true): attention of 128-query tiles over
+// key tiles of kAttnTileKeys rows.  tq: q as [B*H*N, d] bf16 with a 64 x 128
+// box; tk / tv: k / v with a 64 x 4 box (sparse: one 4-token block per box)
+// or a 64 x kAttnTileKeys box (dense tiles).
+constexpr int kAttnTileKeys = 64;
 cudaError_t launch_attention(bool dense, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, const __nv_bfloat16 *k,
                              const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N, int nqb,

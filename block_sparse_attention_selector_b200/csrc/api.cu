@@ -314,7 +314,7 @@ absa_status attention_run(const absa_params *p, const void *q, const void *k, co
     const bool dense = plan == nullptr;
     CUtensorMap tq, tk, tv;
     // sparse gathers: one 4-row box (one 4-token block) per 64-column region
-    const int kv_box = dense ? 128 : 4;
+    const int kv_box = dense ? kAttnTileKeys : 4;
     if (!make_map_bf16(&tq, qh, hr.nbh * p->N, p->d) ||
         !make_map_bf16(&tk, kh, hr.nbh * p->N, p->d, kv_box) ||
         !make_map_bf16(&tv, vh, hr.nbh * p->N, p->d, kv_box))

@@ -6,70 +6,91 @@
 // -ln(pi) (SIP paragraph); the 4-token blocks are gathered by index into
 // full-size tensor-core tiles, tokens are not permuted (third paragraph).
 //
-// Kernel design (one CTA per (b, h, 128-query block), 512 threads):
-//   warps 0-7   softmax, two warpgroups: warpgroup g runs an independent
-//               online softmax over columns 64g..64g+63 of every S tile
-//               (thread = TMEM lane = query row) with its own accumulator
-//               O_g += P_g V_g; the halves are merged in the epilogue
-//   warps 8-14  loaders: TMA gathers of 32 blocks (= 128 key rows) per tile
-//               into SW128 shared-memory tiles; warps 8-10 fill the 2-stage
-//               K ring and the tile's per-column logit bias (4-slot ring),
-//               warps 11-14 the 2-stage V ring, each group at its own pace
-//   warp 15     TMEM owner and MMA issuer (one thread):
-//              S_j = Q K_j^T  -> TMEM (two 128-column buffers)
-//              O_g += P_j[:, 64g..] V_j[64g.., :] -> TMEM (two D-column
-//              accumulators), P_j bf16 in shared memory
+// Kernel design (one CTA per (b, h, 128-query block), 320 threads, about 98 KB
+// of shared memory and 256 TMEM columns, so that two CTAs -- two independent
+// softmax -> P -> PV chains -- share each SM and fill each other's gaps):
+//   warps 0-3   softmax, one warpgroup (thread = TMEM lane = query row) over
+//               all 64 columns of every S tile; it writes P (bf16) back into
+//               the tile's own TMEM columns
+//   warps 4-8   loaders: TMA gathers of 16 blocks (= 64 key rows) per tile into
+//               SW128 shared-memory tiles; warps 4-6 fill the 2-stage K ring
+//               and the tile's per-column logit bias (4-slot ring), warps 7-8
+//               the 2-stage V ring, each group at its own pace
+//   warp 9      TMEM owner and MMA issuer (one thread):
+//               S_j = Q K_j^T  -> TMEM buffer j % 2 (64 columns)
+//               O  += P_j V_j  (A = P_j read from TMEM, B = V_j in shared
+//               memory) -> one D-column accumulator
 // Softmax works in the exp2 domain: x = log2(e) * scale * (q.k) + bias with
-// bias = -log2(pi) for a valid token and -inf for padding; row maxima are
+// bias = -log2(pi) for a valid token and -inf for padding; the row maximum is
 // updated lazily (O is rescaled only when the max grows by more than 2^8), and
 // the final O is divided by the fp32 row sum.
 #include "absa_kernels.cuh"
 
 namespace absa {
 
-template <int D>
-struct AttnSmem {
-    static constexpr int kRegions = D / 64;
-    static constexpr int kTile = 128 * 128;          // one SW128 region of 128 rows
-    static constexpr int kQBytes = kRegions * kTile;
-    static constexpr int kKVBytes = kRegions * kTile;
-    static constexpr int kQOff = 0;
-    static constexpr int kKOff = kQOff + kQBytes;              // [2] stages
-    static constexpr int kVOff = kKOff + 2 * kKVBytes;         // [2] stages
-    static constexpr int kPOff = kVOff + 2 * kKVBytes;         // 128 x 128 bf16
-    static constexpr int kBiasStages = 4;
-    static constexpr int kBiasOff = kPOff + 2 * kTile;         // [4][128] f32
-    static constexpr int kRedOff = kBiasOff + kBiasStages * 128 * 4;  // [2][2][128] f32 final merge
-    static constexpr int kBarOff = kRedOff + 4 * 128 * 4;
-    static constexpr int kBytes = kBarOff + 32 * 8;
-    // keep one CTA per SM so that the 512-column TMEM allocation never waits
-    static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
-};
-
-constexpr int kSoftmaxWarps = 8;              // two warpgroups, 64 columns each
-constexpr int kLoadWarp = kSoftmaxWarps;      // first loader warp
-constexpr int kLoadWarps = 7;                 // warps issuing TMA boxes
-constexpr int kKLoadWarps = 3;                // of which the K group (the rest load V)
-constexpr int kMmaWarp = kLoadWarp + kLoadWarps;   // 15
-constexpr int kAttnThreads = 32 * (kMmaWarp + 1);  // 512
+constexpr int kTileKeys = kAttnTileKeys;               // key rows per tile
+constexpr int kTileBlocks = kTileKeys / 4;             // 4-token blocks per tile
+constexpr int kSoftmaxWarps = 4;                       // one warpgroup
+constexpr int kKLoadWarps = 3;                         // K ring and bias
+constexpr int kVLoadWarps = 2;                         // V ring
+constexpr int kLoadWarp = kSoftmaxWarps;               // first loader warp
+constexpr int kLoadWarps = kKLoadWarps + kVLoadWarps;
+constexpr int kMmaWarp = kLoadWarp + kLoadWarps;       // 9
+constexpr int kAttnThreads = 32 * (kMmaWarp + 1);      // 320
+constexpr int kBiasStages = 4;
+constexpr int kTmemCols = 256;                         // S/P [2][64], O at column 128
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// Loaders.  Sparse mode: a tile's 32 blocks x (d/64) column regions are 4-row
+template <int D>
+struct AttnSmem {
+    static constexpr int kRegions = D / 64;              // 64-element SW128 regions
+    static constexpr int kQRegion = 128 * 128;           // 128 rows of 128 bytes
+    static constexpr int kKVRegion = kTileKeys * 128;    // 64 rows of 128 bytes
+    static constexpr int kQBytes = kRegions * kQRegion;
+    static constexpr int kKVBytes = kRegions * kKVRegion;
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQOff + kQBytes;               // [2] stages
+    static constexpr int kVOff = kKOff + 2 * kKVBytes;          // [2] stages
+    static constexpr int kBiasOff = kVOff + 2 * kKVBytes;       // [4][64] f32
+    static constexpr int kBarOff = kBiasOff + kBiasStages * kTileKeys * 4;
+    static constexpr int kBytes = kBarOff + 32 * 8;
+    static constexpr int kAlloc = kBytes + 1024;  // room to align the tiles to 1024 bytes
+    // the output tile is staged over the (by then idle) K and V rings: rows of
+    // D bf16 with a 16-byte pad against bank conflicts
+    static constexpr int kStageRow = D + 8;
+    static_assert(128 * kStageRow * 2 <= 4 * kKVBytes, "output staging fits the rings");
+};
+
+// O (this thread's TMEM lane, D columns from o_t) *= alpha.  Kept out of line:
+// it runs only when a row maximum grows by more than 2^8, and inlined its
+// registers would add to the softmax loop's.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t o_t, float alpha) {
+#pragma unroll 1
+    for (int ch = 0; ch < D / 16; ++ch) {
+        uint32_t ov[16];
+        tmem_ld16(o_t + ch * 16, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+        tmem_st16(o_t + ch * 16, ov);
+    }
+}
+
+// Loaders.  Sparse mode: a tile's 16 blocks x (d/64) column regions are 4-row
 // TMA boxes (512 bytes each) placed at rows 4i..4i+3 of the SW128 tile; the
 // box swizzle follows the shared-memory address, so a box in the upper half
 // of a 1024-byte atom lands in that half's chunk order.  A group's boxes are
 // spread over its warps (box p goes to warp p % n): a single warp sustains
-// only about 9 bytes/clock of such small boxes, several warps several times
-// that.  Block ids and log(pi) of the next tile are prefetched while the
-// current tile is issued.  Dense mode: one 128-row box per region from one
-// lane.
-// K and V use separate 2-stage rings.  The logit bias of tile t is written
-// together with K_t into slot t % 4 of its own ring (every loader warp arrives
-// on b_full after writing its columns), so the softmax of a tile never waits
-// for that tile's V.
+// only a fraction of the gather rate of several.  Block ids and log(pi) of
+// the next tile are prefetched while the current tile is issued.  Dense
+// mode: one 64-row box per region from one lane.
+// The logit bias of tile t is written together with K_t into slot t % 4 of
+// its own ring (every K loader warp arrives on b_full after writing its
+// columns), so the softmax of a tile never waits for that tile's V.
 template <int D, bool DENSE>
-__global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
+__global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ k,
     const __nv_bfloat16 *__restrict__ v, __nv_bfloat16 *__restrict__ o, int N, int nqb,
@@ -83,19 +104,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     float *bias_s = reinterpret_cast<float *>(sm + S::kBiasOff);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::kBarOff);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;   // [2]
-    uint64_t *k_empty = bars + 3;  // [2]
-    uint64_t *v_full = bars + 5;   // [2]
-    uint64_t *v_empty = bars + 7;  // [2]
-    uint64_t *s_full = bars + 9;   // [2]
-    uint64_t *s_free = bars + 11;  // [2]
-    uint64_t *p_full = bars + 13;  // [2] per column half
-    uint64_t *p_free = bars + 15;  // [2] per column half
-    uint64_t *b_full = bars + 17;  // [4] logit bias of tile j in slot j % 4
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
-    int *bad_flag = reinterpret_cast<int *>(bars + 23);  // a plan entry out of range
-    float *red = reinterpret_cast<float *>(sm + S::kRedOff);  // [max|sum][half][row]
+    uint64_t *k_full = bars + 1;    // [2]
+    uint64_t *k_empty = bars + 3;   // [2]
+    uint64_t *v_full = bars + 5;    // [2]
+    uint64_t *v_empty = bars + 7;   // [2]
+    uint64_t *s_full = bars + 9;    // [2] S_j in TMEM buffer j % 2
+    uint64_t *p_full = bars + 11;   // [2] P_j written over S_j
+    uint64_t *pv_done = bars + 13;  // [2] PV_j complete: buffer j % 2 free, O stable
+    uint64_t *b_full = bars + 15;   // [4] logit bias of tile j in slot j % 4
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
+    int *bad_flag = reinterpret_cast<int *>(bars + 21);  // a plan entry out of range
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -112,18 +131,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             mbar_init(v_full + s, 1);
             mbar_init(v_empty + s, 1);
             mbar_init(s_full + s, 1);
-            mbar_init(s_free + s, kSoftmaxWarps);
+            mbar_init(p_full + s, kSoftmaxWarps);
+            mbar_init(pv_done + s, 1);
         }
-        for (int h = 0; h < 2; ++h) {
-            mbar_init(p_full + h, kSoftmaxWarps / 2);
-            mbar_init(p_free + h, 1);
-        }
-        for (int i = 0; i < S::kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kKLoadWarps);
+        for (int i = 0; i < kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kKLoadWarps);
         *abort_flag = 0;
         *bad_flag = 0;
         mbar_fence_init();
     }
-    if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
 
     // Number of plan entries: a count outside [0, cap] rejects the row (it is
     // written as zeros).  Entries outside [0, NKB) are caught by the loaders,
@@ -139,13 +155,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
             count = 0;
         }
     }
-    const int T = (count + 31) / 32;
+    const int T = (count + kTileBlocks - 1) / kTileBlocks;
     // Rows of a partial tile that no box overwrites must hold finite values
     // (P = 0 there, and 0 * NaN would poison O).  After its first use a ring
     // stage holds finite stale rows, so only a row whose first two tiles are
     // not both full needs the rings cleared (dense tiles past N are zero-filled
     // by the TMA unit).
-    if (!DENSE && count < 64)
+    if (!DENSE && count < 2 * kTileBlocks)
         for (int i = tid; i < 4 * S::kKVBytes / 16; i += kAttnThreads)
             reinterpret_cast<uint4 *>(sm + S::kKOff)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
@@ -154,20 +170,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_o = tmem + 256;  // O_h at tmem_o + 128 h (h = column half)
+    const uint32_t tmem_o = tmem + 128;
 
     if (warp >= kLoadWarp && warp < kLoadWarp + kLoadWarps) {
         // ------------------------------------------------------------ loaders
-        const int lw = warp - kLoadWarp;      // 0..6
+        const int lw = warp - kLoadWarp;      // 0..5
         const bool kside = lw < kKLoadWarps;  // K group (K tiles and bias) or V group
-        const int gw = kside ? lw : lw - kKLoadWarps;              // warp within the group
-        const int gn = kside ? kKLoadWarps : kLoadWarps - kKLoadWarps;  // warps in the group
+        const int gw = kside ? lw : lw - kKLoadWarps;         // warp within the group
+        const int gn = kside ? kKLoadWarps : kVLoadWarps;      // warps in the group
         const int64_t row0 = bh * N;          // first token row of this head
         if (lw == 0 && lane == 0 && T > 0) {
             mbar_arrive_expect_tx(q_full, S::kQBytes);
             const uint32_t q_s = smem_u32(sm + S::kQOff);
             for (int r = 0; r < S::kRegions; ++r)
-                tma_load_2d(q_s + r * S::kTile, &tm_q, 64 * r, (int)(row0 + qb * 128), q_full);
+                tma_load_2d(q_s + r * S::kQRegion, &tm_q, 64 * r, (int)(row0 + qb * 128), q_full);
         }
         const int32_t *idx_row = DENSE ? nullptr : kv_index + row * cap;
         const float *lp_row = DENSE ? nullptr : log_pi + row * cap;
@@ -175,12 +191,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         constexpr int R = S::kRegions;
         const int pbox = gw + gn * lane;
         const int slot = pbox / R, reg = pbox % R;
-        const bool has_box = pbox < 32 * R;
+        const bool has_box = pbox < kTileBlocks * R;
         // this lane's plan entry (block id, log pi) in tile t; -1 past the end
         auto entry = [&](int t, int &b, float &lp) {
             b = -1;
             lp = 0.f;
-            const int e = 32 * t + slot;
+            const int e = kTileBlocks * t + slot;
             if (!DENSE && has_box && e < count) {
                 b = __ldg(idx_row + e);
                 lp = __ldg(lp_row + e);
@@ -190,39 +206,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
         // block 0 instead and marks the row (checked where the entry is used,
         // a tile after its load, so the check adds no load latency).
         auto checked = [&](int t, int b) -> int {
-            if (!DENSE && has_box && 32 * t + slot < count && (b < 0 || b >= nkb)) {
+            if (!DENSE && has_box && kTileBlocks * t + slot < count && (b < 0 || b >= nkb)) {
                 atomicOr(bad_flag, 1);
                 return 0;
             }
             return b;
         };
         // K_t and the logit bias of tile t (bias slot t % 4; a slot is
-        // rewritten only after S_{t-2} has completed, by which time the MMA
-        // order guarantees that tile t-4's softmax is done with it)
+        // rewritten only after S_{t-2} has completed, which the MMA issues
+        // only once PV_{t-4}, and so the softmax of tile t-4, is done)
         auto issue_k = [&](int t, int b, float lpv) -> bool {
             const int st = t & 1;
             b = checked(t, b);
             if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((t - 2) >> 1) & 1,
                                                              status, abort_flag)))
                 return false;
-            float *bias = bias_s + (t % S::kBiasStages) * 128;
+            float *bias = bias_s + (t % kBiasStages) * kTileKeys;
             const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
             if (DENSE) {
                 if (lw == 0) {
-                    float4 bb;
-                    const int t0 = 128 * t + 4 * lane;
+                    float2 bb;
+                    const int t0 = kTileKeys * t + 2 * lane;
                     bb.x = t0 < N ? 0.f : -INFINITY;
                     bb.y = t0 + 1 < N ? 0.f : -INFINITY;
-                    bb.z = t0 + 2 < N ? 0.f : -INFINITY;
-                    bb.w = t0 + 3 < N ? 0.f : -INFINITY;
-                    reinterpret_cast<float4 *>(bias)[lane] = bb;
+                    reinterpret_cast<float2 *>(bias)[lane] = bb;
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(b_full + t % S::kBiasStages);
+                        mbar_arrive(b_full + t % kBiasStages);
                         mbar_arrive_expect_tx(k_full + st, S::kKVBytes);
                         for (int r = 0; r < R; ++r)
-                            tma_load_2d(k_s + r * S::kTile, &tm_k, 64 * r, (int)(row0 + 128 * t),
-                                        k_full + st);
+                            tma_load_2d(k_s + r * S::kKVRegion, &tm_k, 64 * r,
+                                        (int)(row0 + kTileKeys * t), k_full + st);
                     }
                 }
             } else {
@@ -240,11 +254,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(b_full + t % S::kBiasStages);
-                    if (gw == 0) mbar_arrive_expect_tx(k_full + st, min(32, count - 32 * t) * 512 * R);
+                    mbar_arrive(b_full + t % kBiasStages);
+                    if (gw == 0)
+                        mbar_arrive_expect_tx(k_full + st,
+                                              min(kTileBlocks, count - kTileBlocks * t) * 512 * R);
                 }
                 if (b >= 0)
-                    tma_load_2d(k_s + reg * S::kTile + slot * 512, &tm_k, 64 * reg,
+                    tma_load_2d(k_s + reg * S::kKVRegion + slot * 512, &tm_k, 64 * reg,
                                 (int)(row0 + 4 * b), k_full + st);
             }
             return true;
@@ -260,14 +276,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                 if (gw == 0 && lane == 0) {
                     mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
                     for (int r = 0; r < R; ++r)
-                        tma_load_2d(v_s + r * S::kTile, &tm_v, 64 * r, (int)(row0 + 128 * t),
-                                    v_full + st);
+                        tma_load_2d(v_s + r * S::kKVRegion, &tm_v, 64 * r,
+                                    (int)(row0 + kTileKeys * t), v_full + st);
                 }
             } else {
                 if (gw == 0 && lane == 0)
-                    mbar_arrive_expect_tx(v_full + st, min(32, count - 32 * t) * 512 * R);
+                    mbar_arrive_expect_tx(v_full + st,
+                                          min(kTileBlocks, count - kTileBlocks * t) * 512 * R);
                 if (b >= 0)
-                    tma_load_2d(v_s + reg * S::kTile + slot * 512, &tm_v, 64 * reg,
+                    tma_load_2d(v_s + reg * S::kKVRegion + slot * 512, &tm_v, 64 * reg,
                                 (int)(row0 + 4 * b), v_full + st);
             }
             return true;
@@ -287,89 +304,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         // One thread issues, in a fixed order, S_0, S_1 and then for every
-        // tile j: O_0 += P_j[:, 0..63] V_j[0..63, :], O_1 += P_j[:, 64..]
-        // V_j[64.., :], S_{j+2} = Q K_{j+2}^T.  Each step waits (bounded) for
-        // its operands; S_{j+2} also waits for S buffer j % 2 to be read.
+        // tile j: O += P_j V_j, and (once PV_j has completed, so that P_j in
+        // TMEM buffer j % 2 has been read) S_{j+2} = Q K_{j+2}^T into that
+        // buffer.  Each step waits (bounded) for its operands.
         if (lane == 0 && T > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileKeys, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
             const uint32_t q_s = smem_u32(sm + S::kQOff);
-            const uint32_t p_s = smem_u32(sm + S::kPOff);
             auto issue_s = [&](int js) -> bool {
                 const int st = js & 1;
                 if (!mbar_wait(k_full + st, (js >> 1) & 1, status, abort_flag)) return false;
-                if (js >= 2 && !mbar_wait(s_free + st, ((js - 2) >> 1) & 1, status, abort_flag))
-                    return false;
                 tc_fence_after();
                 const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * S::kTile + (ks & 3) * 32;
-                    tc_mma_f16(tmem + st * 128, sw128_desc(q_s + off, 16, 1024),
-                               sw128_desc(k_s + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                    const uint32_t qoff = (ks >> 2) * S::kQRegion + (ks & 3) * 32;
+                    const uint32_t koff = (ks >> 2) * S::kKVRegion + (ks & 3) * 32;
+                    tc_mma_f16(tmem + st * kTileKeys, sw128_desc(q_s + qoff, 16, 1024),
+                               sw128_desc(k_s + koff, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                 }
                 tc_commit(s_full + st);
                 tc_commit(k_empty + st);
                 return true;
             };
-            auto issue_pv = [&](int j, int h) -> bool {
+            auto issue_pv = [&](int j) -> bool {
                 const int st = j & 1;
-                if (!mbar_wait(p_full + h, j & 1, status, abort_flag)) return false;
-                if (h == 0 && !mbar_wait(v_full + st, (j >> 1) & 1, status, abort_flag)) return false;
+                if (!mbar_wait(p_full + st, (j >> 1) & 1, status, abort_flag)) return false;
+                if (!mbar_wait(v_full + st, (j >> 1) & 1, status, abort_flag)) return false;
                 tc_fence_after();
-                // O_h += P[:, 64h .. 64h+63] V[64h .. 64h+63, :]
                 const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = sw128_desc(p_s + h * S::kTile + ks * 32, 16, 1024);
-                    const uint64_t bdesc = sw128_desc(v_s + (64 * h + 16 * ks) * 128, S::kTile, 1024);
-                    tc_mma_f16(tmem_o + 128 * h, a, bdesc, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < kTileKeys / 16; ++ks) {  // 16 keys = 8 P columns per step
+                    const uint64_t bdesc =
+                        sw128_desc(v_s + (16 * ks) * 128, S::kKVRegion, 1024);
+                    tc_mma_f16_tmem_a(tmem_o, tmem + st * kTileKeys + 8 * ks, bdesc, idesc_o,
+                                      (j > 0 || ks > 0) ? 1u : 0u);
                 }
-                tc_commit(p_free + h);
-                if (h == 1) tc_commit(v_empty + st);  // both halves of tile j issued
+                tc_commit(pv_done + st);
+                tc_commit(v_empty + st);
                 return true;
             };
             bool ok = mbar_wait(q_full, 0, status, abort_flag) && issue_s(0);
             if (ok && T > 1) ok = issue_s(1);
             for (int j = 0; j < T && ok; ++j) {
-                ok = issue_pv(j, 0) && issue_pv(j, 1);
-                if (ok && j + 2 < T) ok = issue_s(j + 2);
+                ok = issue_pv(j);
+                if (ok && j + 2 < T)
+                    ok = mbar_wait(pv_done + (j & 1), (j >> 1) & 1, status, abort_flag) &&
+                         issue_s(j + 2);
             }
         }
     } else {
         // ------------------------------------------------------------- softmax
-        // Warpgroup `half` runs its own online softmax over columns
-        // 64*half .. 64*half+63 of every S tile, with its own running max,
-        // row sum and accumulator O_half (O_half += P_half V_half); the two
-        // halves are merged in the epilogue, so no per-tile exchange is
-        // needed.  Thread = TMEM lane = query row.
-        const int half = warp >> 2;
-        const int r = (warp & 3) * 32 + lane;  // query row = TMEM lane
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t p_s = smem_u32(sm + S::kPOff) + half * S::kTile;
-        const int cb = 64 * half;
-        const uint32_t o_h = tmem_o + 128 * half + lane_base;
+        // Thread = TMEM lane = query row; one online softmax over the 64
+        // columns of every S tile.  P_j (bf16) goes into the first 32 columns
+        // of S_j's own TMEM buffer (two keys per column), where the PV MMA
+        // reads it.
+        const int r = warp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t o_t = tmem_o + lane_base;
         float m_ref = -INFINITY, lsum = 0.f;
         bool ok = true;
         for (int j = 0; j < T; ++j) {
             const int b = j & 1;
+            const uint32_t s_t = tmem + lane_base + b * kTileKeys;
             ok = __all_sync(0xffffffffu, mbar_wait(s_full + b, (j >> 1) & 1, status, abort_flag));
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[2][32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-                tmem_ld32(tmem + lane_base + b * 128 + cb + ch * 32, sv[ch]);
+            tmem_ld32(s_t, sv[0]);
+            tmem_ld32(s_t + 32, sv[1]);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_free + b);
-            const int bs = j % S::kBiasStages;
-            ok = __all_sync(0xffffffffu, mbar_wait(b_full + bs, (j / S::kBiasStages) & 1, status, abort_flag));
+            const int bs = j % kBiasStages;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(b_full + bs, (j / kBiasStages) & 1, status, abort_flag));
             if (!ok) break;
-            const uint32_t bias_u = smem_u32(bias_s + bs * 128 + cb);
+            const uint32_t bias_u = smem_u32(bias_s + bs * kTileKeys);
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            const uint64_t sc2 = ((uint64_t)__float_as_uint(scale_log2) << 32) | __float_as_uint(scale_log2);
+            const uint64_t sc2 =
+                ((uint64_t)__float_as_uint(scale_log2) << 32) | __float_as_uint(scale_log2);
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
@@ -378,124 +390,96 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
                     asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
                                  : "=l"(b01), "=l"(b23)
                                  : "r"(bias_u + (uint32_t)(ch * 32 + i) * 4u));
-                    const uint64_t x01 = f32x2_fma(((uint64_t)sv[ch][i + 1] << 32) | sv[ch][i], sc2, b01);
-                    const uint64_t x23 = f32x2_fma(((uint64_t)sv[ch][i + 3] << 32) | sv[ch][i + 2], sc2, b23);
+                    const uint64_t x01 =
+                        f32x2_fma(((uint64_t)sv[ch][i + 1] << 32) | sv[ch][i], sc2, b01);
+                    const uint64_t x23 =
+                        f32x2_fma(((uint64_t)sv[ch][i + 3] << 32) | sv[ch][i + 2], sc2, b23);
                     sv[ch][i] = (uint32_t)x01;
                     sv[ch][i + 1] = (uint32_t)(x01 >> 32);
                     sv[ch][i + 2] = (uint32_t)x23;
                     sv[ch][i + 3] = (uint32_t)(x23 >> 32);
                     const int a = (i >> 2) & 3;
-                    mx4[a] = fmaxf(mx4[a], fmaxf(fmaxf(__uint_as_float(sv[ch][i]), __uint_as_float(sv[ch][i + 1])),
-                                                 fmaxf(__uint_as_float(sv[ch][i + 2]), __uint_as_float(sv[ch][i + 3]))));
+                    mx4[a] = fmaxf(mx4[a],
+                                   fmaxf(fmaxf(__uint_as_float(sv[ch][i]), __uint_as_float(sv[ch][i + 1])),
+                                         fmaxf(__uint_as_float(sv[ch][i + 2]), __uint_as_float(sv[ch][i + 3]))));
                 }
             const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             // lazy max: keep the reference unless the tile exceeds it by 2^8;
-            // a half whose columns so far were all padding has m_ref = -inf
-            const bool need = tmax > m_ref + kRescaleThreshold || (m_ref == -INFINITY && tmax > -INFINITY);
+            // a row whose columns so far were all padding has m_ref = -inf
+            const bool need =
+                tmax > m_ref + kRescaleThreshold || (m_ref == -INFINITY && tmax > -INFINITY);
             const bool any_need = j > 0 && __any_sync(0xffffffffu, need);
             const float m_new = need ? tmax : m_ref;
             const float alpha = m_ref == -INFINITY ? 0.f : ex2(m_ref - m_new);
             m_ref = m_new;
-            if (j >= 1) {  // PV of this half's previous tile is done: P half free, O_half stable
-                ok = __all_sync(0xffffffffu, mbar_wait(p_free + half, (j - 1) & 1, status, abort_flag));
-                if (!ok) break;
-            }
             const float moff = m_ref == -INFINITY ? 0.f : -m_ref;
             const uint64_t moff2 = ((uint64_t)__float_as_uint(moff) << 32) | __float_as_uint(moff);
             uint64_t acc2[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {  // P_j in two halves of 16 columns (32 keys)
+                uint32_t pk[16];
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {  // 8 columns = one 16-byte chunk
-                    float p[8];
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const uint64_t y2 = f32x2_add(((uint64_t)sv[ch][g * 8 + e + 1] << 32) | sv[ch][g * 8 + e], moff2);
-                        p[e] = ex2(__uint_as_float((uint32_t)y2));
-                        p[e + 1] = ex2(__uint_as_float((uint32_t)(y2 >> 32)));
-                        acc2[e >> 1] = f32x2_add(acc2[e >> 1], ((uint64_t)__float_as_uint(p[e + 1]) << 32) | __float_as_uint(p[e]));
-                    }
-                    const uint32_t dst = p_s + sw128_offset(r, ch * 4 + g);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                                 "r"(pack_bf16x2(p[0], p[1])), "r"(pack_bf16x2(p[2], p[3])),
-                                 "r"(pack_bf16x2(p[4], p[5])), "r"(pack_bf16x2(p[6], p[7]))
-                                 : "memory");
+                for (int e = 0; e < 32; e += 2) {
+                    const uint64_t y2 =
+                        f32x2_add(((uint64_t)sv[ch][e + 1] << 32) | sv[ch][e], moff2);
+                    const float p0 = ex2(__uint_as_float((uint32_t)y2));
+                    const float p1 = ex2(__uint_as_float((uint32_t)(y2 >> 32)));
+                    acc2[(e >> 1) & 3] = f32x2_add(acc2[(e >> 1) & 3],
+                                                   ((uint64_t)__float_as_uint(p1) << 32) | __float_as_uint(p0));
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
                 }
+                tmem_st16(s_t + 16 * ch, pk);
             }
-            if (any_need) {  // lazy rescale of O_half by exp2(m_old - m_new)
-                tc_fence_after();
-                lsum *= alpha;
-#pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t ov[32];
-                    tmem_ld32(o_h + ch * 32, ov);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(o_h + ch * 32, ov);
-                }
-                tmem_wait_st();
-            }
+            float tsum;
             {
                 const uint64_t a01 = f32x2_add(acc2[0], acc2[1]), a23 = f32x2_add(acc2[2], acc2[3]);
                 const uint64_t a = f32x2_add(a01, a23);
-                lsum += __uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)(a >> 32));
+                tsum = __uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)(a >> 32));
             }
-            fence_proxy_async_smem();
+            if (any_need) {  // lazy rescale of O by exp2(m_old - m_new) once PV_{j-1} is done
+                ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1,
+                                                       status, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                lsum *= alpha;
+                rescale_o<D>(o_t, alpha);
+            }
+            lsum += tsum;
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + half);
+            if (lane == 0) mbar_arrive(p_full + b);
         }
-        // epilogue: o = (O_0 a_0 + O_1 a_1) / (l_0 a_0 + l_1 a_1), a_h = 2^(m_h - max);
-        // warpgroup `half` writes output columns (D/2) half .. (D/2) half + D/2 - 1.
-        // Every softmax thread reaches this barrier exactly once.
-        red[half * 128 + r] = m_ref;
-        red[256 + half * 128 + r] = lsum;
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
-        const float m0 = red[r], m1 = red[128 + r];
-        const float mm = fmaxf(m0, m1);
-        const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
-        const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
-        const float ltot = red[256 + r] * a0 + red[384 + r] * a1;
-        constexpr int OC = D / 2;
-        // The output tile goes through shared memory (the K ring, idle by now:
-        // every K tile has been consumed) so that the global stores are
-        // coalesced: rows of D bf16 with a 16-byte pad against bank conflicts.
-        constexpr int kStageRow = D + 8;
+        // epilogue: o = O / l.  Every softmax thread reaches the barriers below
+        // exactly once.
+        constexpr int kStageRow = S::kStageRow;
         __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + S::kKOff);
         // a plan entry out of range (seen by the loaders before their last
         // arrival on b_full, which every softmax warp has waited for)
         const bool bad_row = !DENSE && T > 0 && *reinterpret_cast<volatile int *>(bad_flag) != 0;
-        if (T > 0 && ok && !bad_row) {
-            ok = __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, status, abort_flag) &&
-                                             mbar_wait(p_free + 1, (T - 1) & 1, status, abort_flag));
-        }
+        if (T > 0 && ok && !bad_row)
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1,
+                                                   status, abort_flag));
         const bool write = T > 0 && ok && !bad_row;
         if (write) {
+            // the last PV has completed, and with it every MMA that read the
+            // rings; every TMA copy into them has been waited for
             tc_fence_after();
-            fence_proxy_async_smem();  // generic writes after the ring's async-proxy use
-            const float inv = 1.f / ltot;
-            const float c0 = a0 * inv, c1 = a1 * inv;
-#pragma unroll
-            for (int ch = 0; ch < OC / 32; ++ch) {
-                uint32_t o0[32], o1[32];
-                tmem_ld32(tmem_o + lane_base + half * OC + ch * 32, o0);
-                tmem_ld32(tmem_o + 128 + lane_base + half * OC + ch * 32, o1);
+            fence_proxy_async_smem();  // generic writes after the rings' async-proxy use
+            const float inv = 1.f / lsum;
+#pragma unroll 1
+            for (int ch = 0; ch < D / 16; ++ch) {
+                uint32_t ov[16];
+                tmem_ld16(o_t + ch * 16, ov);
                 tmem_wait_ld();
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        f[e] = __uint_as_float(o0[8 * g + e]) * c0 +
-                               __uint_as_float(o1[8 * g + e]) * c1;
+                for (int g = 0; g < 2; ++g) {
                     uint4 u;
-                    u.x = pack_bf16x2(f[0], f[1]);
-                    u.y = pack_bf16x2(f[2], f[3]);
-                    u.z = pack_bf16x2(f[4], f[5]);
-                    u.w = pack_bf16x2(f[6], f[7]);
-                    *reinterpret_cast<uint4 *>(stage + r * kStageRow + half * OC + ch * 32 + 8 * g) = u;
+                    u.x = pack_bf16x2(__uint_as_float(ov[8 * g]) * inv, __uint_as_float(ov[8 * g + 1]) * inv);
+                    u.y = pack_bf16x2(__uint_as_float(ov[8 * g + 2]) * inv, __uint_as_float(ov[8 * g + 3]) * inv);
+                    u.z = pack_bf16x2(__uint_as_float(ov[8 * g + 4]) * inv, __uint_as_float(ov[8 * g + 5]) * inv);
+                    u.w = pack_bf16x2(__uint_as_float(ov[8 * g + 6]) * inv, __uint_as_float(ov[8 * g + 7]) * inv);
+                    *reinterpret_cast<uint4 *>(stage + r * kStageRow + ch * 16 + 8 * g) = u;
                 }
             }
         }
@@ -515,7 +499,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) absa_attention_kernel(
     if (warp == kMmaWarp) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -529,6 +513,11 @@ static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &
     const int smem = AttnSmem<D>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // two CTAs per SM: ask for the largest shared-memory carveout
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     absa_attention_kernel<D, DENSE><<<(unsigned)(BH * nqb), kAttnThreads, smem, stream>>>(
         tq, tk, tv, k, v, o, N, nqb, nkb, scale_log2, counts, kv_index, log_pi, cap, status);

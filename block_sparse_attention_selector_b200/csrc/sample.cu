@@ -80,9 +80,11 @@ __device__ __forceinline__ void block_sum2(uint64_t &a, int &b, uint64_t *red_a,
     }
 }
 
-// Shared-memory lists of a plan row.
+// Shared-memory state of a plan row.
 constexpr int kSampleCand = 2048;  // q - 1 of the blocks at or above the list threshold
-constexpr int kSampleList = 4096;  // q - 1 of the first written entries (for the ln(pi) pass)
+// Iterations of 128 blocks (32 chunks of 4) in the longest row (the row start
+// may sit up to 3 blocks before a 16-byte boundary).
+constexpr int kSampleMaxIters = (kSampleMaxKvBlocks + 3 + 127) / 128;
 
 // Scores of a row as 16-byte chunks: chunk c holds blocks 4c - off .. 4c - off + 3,
 // where off (0..3) aligns the row start to 16 bytes; blocks outside [0, nkb)
@@ -124,15 +126,20 @@ __device__ __forceinline__ float f4_get(const float4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// Warp-wide sum mod R (every lane gets it).
+__device__ __forceinline__ uint64_t warp_sum_mod(uint64_t x, uint64_t R) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = addmod(x, __shfl_xor_sync(0xffffffffu, x, o), R);
+    return x;
+}
+
 // One CTA per plan row (b,h,qb); the grid covers rows row0 .. row0+gridDim-1
 // of the whole problem (scores and plan pointers start at row0, the draw
-// counter uses the global row).  The row is walked in tiles of 4 * threads
-// consecutive key blocks (thread t: the 4 blocks of chunk tile*threads + t),
-// three times:
+// counter uses the global row).
 //  A  (from memory) q_j - 1 = quantised score, R0 = sum_j q_j, and the list of
 //     q_j at or above t_list = ceil(2^30 / n) (for scores summing to about 1 that
 //     is a quarter of the first capping threshold R0 / n, a few hundred blocks
-//     on the workloads).
+//     on the workloads), in tiles of 4 * threads consecutive blocks.
 //  -  Capping rounds of the definition: C_{t+1} = {j : r_t q_j >= R_t} with
 //     r_t = n - |C_t|, R_t = R0 - sum_{C_t} q_j, from C_0 = {} until |C| stops
 //     growing.  Every capped set contains the previous one, so each round is a
@@ -141,12 +148,23 @@ __device__ __forceinline__ float f4_get(const float4 &v, int i) {
 //     are then listed), and otherwise (or if the list overflowed) over the
 //     whole row from memory.  At the fixed point, j is capped iff
 //     r* q_j >= R*.
-//  C  (from memory again; the row is still in L2) the draws and an ascending
-//     compaction: per tile, a CTA-wide scan of the per-thread taken counts
-//     places every taken block; its q - 1 goes to a shared list for the last
-//     pass.
-//  -  ln(pi) of the written entries, all threads busy (the double-precision
-//     logarithm would otherwise run once per taken lane of every warp step).
+//  C  (from memory again; the row is still in L2) the take decision of every
+//     block: warp w walks its own contiguous segment of the row, 128 blocks
+//     (a 16-byte chunk per lane) per step, and keeps four ballots of take bits
+//     per step in shared memory.
+//  -  Compaction: one scan of the warps' counts places each segment; the warp
+//     walks its ballots again and writes its taken block ids in ascending
+//     order.
+//  -  ln(pi) of the written entries (their scores re-read by id), all threads
+//     busy (the double-precision logarithm would otherwise run once per taken
+//     lane of every warp step).
+// Poisson draws are decided in fp32 first: with x = u/2^32 and the uncapped
+// pi_j = r q_j / R, the block is taken iff x < pi_j.  d = x' - s' K with
+// x' = x truncated to 23 bits, s' = s clamped to [0, 1] (NaN -> 0) and
+// K = fl(r 2^32 / R) differs from x - pi_j by at most r/R (|q - s' 2^32| <= 1)
+// plus 2^-21.7 of rounding, so |d| > r/R + 2^-20 decides exactly (a capped
+// block, pi_j >= 1, always gives d < 0 or lands in the margin); the blocks
+// within the margin take the exact integer test.
 template <int WARPS>
 __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_kernel(
     const float *__restrict__ scores, int nkb, int64_t n, uint64_t seed, int cap,
@@ -154,11 +172,11 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
     uint64_t *__restrict__ r_R, int32_t *status, int64_t row0, int design, int nqb) {
     constexpr int kThreads = 32 * WARPS;
     __shared__ uint32_t cand[kSampleCand];
-    __shared__ uint32_t list[kSampleList];
+    __shared__ uint4 takew[kSampleMaxIters];  // per step: ballots of take bit i of each lane
     __shared__ uint64_t red_a[WARPS];
     __shared__ int red_b[WARPS];
-    __shared__ int wcnt[2][WARPS];
-    __shared__ uint64_t wmod[2][WARPS];
+    __shared__ int wcnt[WARPS];
+    __shared__ uint64_t wmod[WARPS];
     __shared__ int n_cand;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -267,7 +285,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
     const uint32_t r32 = (uint32_t)r;  // 1 <= r <= n < NKB < 2^16
     const uint32_t Rh = (uint32_t)(R >> 32), Rl = (uint32_t)R;
 
-    // ---- pass C: draws and ascending compaction
+    // ---- pass C: take bits of this warp's segment
     // SplitMix64 state of block j is base + j * gamma with
     // base = mix(seed) + (draw row * NKB + 1) * gamma; the draw row is the
     // global row, or under the paired design that of the even query block of
@@ -276,111 +294,149 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
     const int64_t drow =
         row0 + row - (design == ABSA_SAMPLING_PAIRED ? (int)(blockIdx.x % (unsigned)nqb) & 1 : 0);
     const uint64_t base = splitmix64_mix(seed) + ((uint64_t)drow * (uint64_t)nkb + 1) * kGamma;
-    const bool systematic = design == ABSA_SAMPLING_SYSTEMATIC;
-    // Systematic design.  Interval j is [A_j, A_j + a_j) with a_j = R on C and
-    // r q_j elsewhere, A_j = sum_{i<j} a_i; the points are (k + U/2^32) R.
-    // With rho_j = A_j mod R (capped blocks add 0 mod R) and
-    // F = floor(U R / 2^32), an uncapped interval (a_j < R) holds the point of
-    // its own period iff rho_j <= F < rho_j + a_j and that of the next period
-    // iff R + F < rho_j + a_j (comparisons of the exact values U R vs multiples
-    // of 2^32 reduce to these on F).  rho comes from a CTA-wide scan mod R per
-    // tile, carried across tiles.
-    uint64_t F = 0;
-    if (systematic) {
-        const uint32_t U = splitmix64_hi32(base);  // the draw of block 0 of the row
-        F = (uint64_t)U * Rh + __umulhi(U, Rl);
-    }
-    uint64_t rho_carry = 0;
-    int total = 0;
-    float4 v = sr.chunk(tid);
-    for (int t = 0; t < ntiles; ++t) {
-        const int ch = t * kThreads + tid;
-        const float4 vn = sr.chunk(ch + kThreads);  // next tile, in flight during this one
-        const uint32_t valid = sr.valid_mask(ch);
-        const int j0 = 4 * ch - sr.off;
-        uint32_t qm[4];
-        uint64_t rq[4];
-        uint32_t capped = 0;
+    const int niters = (sr.nchunks + 31) >> 5;
+    const int per = (niters + WARPS - 1) / WARPS;
+    const int i0 = min(niters, warp * per), i1 = min(niters, i0 + per);
+    const uint32_t below = (1u << lane) - 1u;
+    int wtaken = 0;  // taken blocks of this warp's segment
+    // exact take bits of the 4 blocks of chunk c (capped, or the exact draw)
+    auto exact_bits = [&](const float4 &v, uint64_t st, uint32_t which) -> uint32_t {
+        uint32_t bits = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            qm[i] = quantise_m1(f4_get(v, i));
-            rq[i] = (uint64_t)r32 * qm[i] + r32;
-            if (((valid >> i) & 1u) && rq[i] >= R) capped |= 1u << i;
-        }
-        uint32_t bits = capped;
-        if (!systematic) {
-            uint64_t state = base + (uint64_t)(int64_t)j0 * kGamma;
-#pragma unroll
-            for (int i = 0; i < 4; ++i, state += kGamma)
-                if (((valid & ~capped) >> i) & 1u)
-                    bits |= draw_taken(splitmix64_hi32(state), Rh, Rl, rq[i]) ? 1u << i : 0u;
-        } else {
-            uint64_t e[4], lsum = 0;
+        for (int i = 0; i < 4; ++i)
+            if ((which >> i) & 1u) {
+                const uint64_t rq = (uint64_t)r32 * quantise_m1(f4_get(v, i)) + r32;
+                if (rq >= R || draw_taken(splitmix64_hi32(st + (uint64_t)i * kGamma), Rh, Rl, rq))
+                    bits |= 1u << i;
+            }
+        return bits;
+    };
+    auto store_bits = [&](int it, uint32_t bits) {
+        const uint32_t b0 = __ballot_sync(0xffffffffu, bits & 1u);
+        const uint32_t b1 = __ballot_sync(0xffffffffu, bits & 2u);
+        const uint32_t b2 = __ballot_sync(0xffffffffu, bits & 4u);
+        const uint32_t b3 = __ballot_sync(0xffffffffu, bits & 8u);
+        if (lane == 0) takew[it] = make_uint4(b0, b1, b2, b3);
+        wtaken += __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
+    };
+    if (design != ABSA_SAMPLING_SYSTEMATIC) {
+        const float K = (float)((double)r * 4294967296.0 / (double)R);
+        const float margin = (float)((double)r / (double)R) + 0x1p-20f;
+        uint64_t st = base + (uint64_t)(int64_t)(4 * (i0 * 32 + lane) - sr.off) * kGamma;
+        for (int it = i0; it < i1; ++it, st += 128 * kGamma) {
+            const int c = it * 32 + lane;
+            const float4 v = sr.chunk(c);
+            const uint32_t valid = sr.valid_mask(c);
+            uint32_t bits = 0, near = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                e[i] = (((valid & ~capped) >> i) & 1u) ? rq[i] : 0;  // a_j mod R
-                lsum = addmod(lsum, e[i], R);
+                const uint32_t u = splitmix64_hi32(st + (uint64_t)i * kGamma);
+                const float x = __uint_as_float((u >> 9) | 0x3F800000u) - 1.0f;
+                const float s = fminf(fmaxf(f4_get(v, i), 0.f), 1.f);  // NaN -> 0
+                const float d = __fmaf_rn(-s, K, x);
+                bits |= d < 0.f ? 1u << i : 0u;
+                near |= fabsf(d) <= margin ? 1u << i : 0u;
             }
-            uint64_t inc = lsum;  // inclusive warp scan mod R
+            near &= valid;
+            if (__any_sync(0xffffffffu, near != 0))  // rare: exact test near the threshold
+                bits = (bits & ~near) | exact_bits(v, st, near);
+            store_bits(it, bits & valid);
+        }
+    } else {
+        // Systematic design.  Interval j is [A_j, A_j + a_j) with a_j = R on
+        // C and r q_j elsewhere, A_j = sum_{i<j} a_i; the points are
+        // (k + U/2^32) R.  With rho_j = A_j mod R (capped blocks add 0 mod R)
+        // and F = floor(U R / 2^32), an uncapped interval (a_j < R) holds the
+        // point of its own period iff rho_j <= F < rho_j + a_j and that of the
+        // next period iff R + F < rho_j + a_j (comparisons of the exact values
+        // U R vs multiples of 2^32 reduce to these on F).  rho comes from the
+        // segment totals (first sweep, one scan over the warps) and a warp
+        // scan mod R per step (second sweep).
+        const uint32_t U = splitmix64_hi32(base);  // the draw of block 0 of the row
+        const uint64_t F = (uint64_t)U * Rh + __umulhi(U, Rl);
+        // a_j mod R of a chunk's 4 blocks (0 when capped or outside the row)
+        auto elems = [&](int c, uint64_t (&e)[4], uint32_t &capped) {
+            const float4 v = sr.chunk(c);
+            const uint32_t valid = sr.valid_mask(c);
+            capped = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint64_t rq = (uint64_t)r32 * quantise_m1(f4_get(v, i)) + r32;
+                const bool in = (valid >> i) & 1u;
+                if (in && rq >= R) capped |= 1u << i;
+                e[i] = (in && rq < R) ? rq : 0;
+            }
+        };
+        uint64_t seg = 0;
+        for (int it = i0; it < i1; ++it) {
+            uint64_t e[4];
+            uint32_t cb;
+            elems(it * 32 + lane, e, cb);
+            uint64_t ls = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ls = addmod(ls, e[i], R);
+            seg = addmod(seg, warp_sum_mod(ls, R), R);
+        }
+        if (lane == 0) wmod[warp] = seg;
+        __syncthreads();
+        uint64_t rho0 = 0;  // rho of this segment's first block
+        for (int w = 0; w < warp; ++w) rho0 = addmod(rho0, wmod[w], R);
+        for (int it = i0; it < i1; ++it) {
+            uint64_t e[4];
+            uint32_t bits;
+            elems(it * 32 + lane, e, bits);
+            uint64_t ls = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ls = addmod(ls, e[i], R);
+            uint64_t inc = ls;  // inclusive warp scan mod R
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc = addmod(inc, y, R);
             }
-            if (lane == 31) wmod[t & 1][warp] = inc;
-            __syncthreads();
-            uint64_t rho = rho_carry, tile_sum = 0;
-#pragma unroll
-            for (int w = 0; w < WARPS; ++w) {
-                const uint64_t x = wmod[t & 1][w];
-                if (w < warp) rho = addmod(rho, x, R);
-                tile_sum = addmod(tile_sum, x, R);
-            }
-            rho = addmod(rho, submod(inc, lsum, R), R);
-            rho_carry = addmod(rho_carry, tile_sum, R);
+            uint64_t rho = addmod(rho0, submod(inc, ls, R), R);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint64_t a = e[i];
                 if (a != 0 && ((rho <= F && F < rho + a) || R + F < rho + a)) bits |= 1u << i;
                 rho = addmod(rho, a, R);
             }
+            rho0 = addmod(rho0, __shfl_sync(0xffffffffu, inc, 31), R);
+            store_bits(it, bits);
         }
-        // CTA-wide exclusive scan of the taken counts
-        const int cnt = __popc(bits);
-        int inc = cnt;
+    }
+
+    // ---- compaction: segments in warp order, ascending blocks within each
+    if (lane == 0) wcnt[warp] = wtaken;
+    __syncthreads();
+    int pos = 0, total = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
-        }
-        if (lane == 31) wcnt[t & 1][warp] = inc;
-        __syncthreads();
-        int pos = total, tile_total = 0;
-#pragma unroll
-        for (int w = 0; w < WARPS; ++w) {
-            const int x = wcnt[t & 1][w];
-            pos += w < warp ? x : 0;
-            tile_total += x;
-        }
-        pos += inc - cnt;
+    for (int w = 0; w < WARPS; ++w) {
+        const int x = wcnt[w];
+        pos += w < warp ? x : 0;
+        total += x;
+    }
+    for (int it = i0; it < i1 && pos < cap; ++it) {
+        const uint4 W = takew[it];
+        const uint32_t nib = ((W.x >> lane) & 1u) | (((W.y >> lane) & 1u) << 1) |
+                             (((W.z >> lane) & 1u) << 2) | (((W.w >> lane) & 1u) << 3);
+        int p = pos + __popc(W.x & below) + __popc(W.y & below) + __popc(W.z & below) +
+                __popc(W.w & below);
+        const int j0 = 4 * (it * 32 + lane) - sr.off;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            if ((bits >> i) & 1u) {
-                if (pos < cap) {
-                    idx_row[pos] = j0 + i;
-                    if (pos < kSampleList) list[pos] = qm[i];
-                }
-                ++pos;
+            if ((nib >> i) & 1u) {
+                if (p < cap) idx_row[p] = j0 + i;
+                ++p;
             }
-        total += tile_total;
-        v = vn;
+        pos += __popc(W.x) + __popc(W.y) + __popc(W.z) + __popc(W.w);
     }
-    __syncthreads();  // list and the kv_index entries are visible to the whole CTA
+    __syncthreads();  // the kv_index entries written above are visible to the whole CTA
 
     // ---- ln(pi) of the written entries
     const int written = min(total, cap);
     for (int p = tid; p < written; p += kThreads) {
-        const uint32_t qmp = p < kSampleList ? list[p] : quantise_m1(__ldg(srow + idx_row[p]));
+        const uint32_t qmp = quantise_m1(__ldg(srow + idx_row[p]));
         const uint64_t rqp = (uint64_t)r32 * qmp + r32;
         lp_row[p] = rqp >= R ? 0.f : (float)log((double)rqp / (double)R);
     }
