@@ -78,14 +78,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // Wait for the phase with the given parity.  Returns false (after setting the
 // timeout flag in *status and *abort) if it does not complete within about
 // limit_cycles SM clocks, or if another thread of the CTA already gave up.
-// After a short poll the thread sleeps between checks; the clock and the
-// abort flag are read once every 16 sleeps so that waiting warps take few
-// issue slots.
+// `polls` non-blocking probes come first: a latency-critical waiter (most of
+// its waits end within a few hundred cycles, and a sleeping thread wakes up
+// late) polls; a waiter that is normally ahead of its producer (a loader)
+// sleeps at once and leaves the issue slots to the warps doing the math.
+// Then the thread sleeps between checks; the clock and the abort flag are
+// read once every 16 sleeps so that waiting warps take few issue slots.
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, int32_t *status,
-                                                volatile int *abort, long long limit_cycles) {
-    // short non-blocking poll first: most waits end within a few hundred cycles
-    // and a sleeping thread wakes up late
-    for (int i = 0; i < 64; ++i)
+                                                volatile int *abort, long long limit_cycles,
+                                                int polls = 64) {
+    for (int i = 0; i < polls; ++i)
         if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t i = 1;; ++i) {
@@ -103,8 +105,8 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, 
 
 // mbar_wait_limit with the library's limit (kWaitLimitCycles, about a second).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
-                                          volatile int *abort) {
-    return mbar_wait_limit(bar, parity, status, abort, kWaitLimitCycles);
+                                          volatile int *abort, int polls = 64) {
+    return mbar_wait_limit(bar, parity, status, abort, kWaitLimitCycles, polls);
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
@@ -284,26 +286,6 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x on the FMA pipe, for x <= 0 (x below -125, -inf included, gives
-// 2^-125 instead of 0).  Range reduction x = n + f with n = round(x) from the
-// 1.5 * 2^23 rounding constant and f in [-1/2, 1/2]; 2^f from a degree-4
-// polynomial fitted here for relative error over [-1/2, 1/2] (maximum
-// relative error 2.7e-6 in fp32 Horner form); 2^n is added to the exponent
-// field (n is the low bits of the rounded sum, whose constant has zero low
-// 9 bits, so a 23-bit shift of its bit pattern is n << 23).  Used for part
-// of the exponentials where the MUFU unit is the limit and an error of a few
-// 1e-6 is far inside the tolerance.
-__device__ __forceinline__ float ex2_fma(float x) {
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    float p = __fmaf_rn(0.009570378810167313f, f, 0.05591868609189987f);
-    p = __fmaf_rn(p, f, 0.240247443318367f);
-    p = __fmaf_rn(p, f, 0.6931216716766357f);
-    p = __fmaf_rn(p, f, 0.9999992847442627f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // Two fp32 lanes per instruction (each lane rounds like the scalar op).

@@ -38,6 +38,7 @@ constexpr int kLoadWarps = kKLoadWarps + kVLoadWarps;
 constexpr int kMmaWarp = kLoadWarp + kLoadWarps;       // 9
 constexpr int kAttnThreads = 32 * (kMmaWarp + 1);      // 320
 constexpr int kBiasStages = 4;
+constexpr int kLoaderPolls = 0;                        // loaders sleep at once when they wait
 constexpr int kTmemCols = 256;                         // S/P [2][64], O at column 128
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             const int st = t & 1;
             b = checked(t, b);
             if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((t - 2) >> 1) & 1,
-                                                             status, abort_flag)))
+                                                             status, abort_flag, kLoaderPolls)))
                 return false;
             float *bias = bias_s + (t % kBiasStages) * kTileKeys;
             const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             const int st = t & 1;
             b = checked(t, b);
             if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(v_empty + st, ((t - 2) >> 1) & 1,
-                                                             status, abort_flag)))
+                                                             status, abort_flag, kLoaderPolls)))
                 return false;
             const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
             if (DENSE) {

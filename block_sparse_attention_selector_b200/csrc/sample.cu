@@ -32,11 +32,16 @@ constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;  // SplitMix64 increment
 // z = hi 2^32 + lo, the high word of z * c mod 2^64 is
 // hi32(lo * c_lo) + lo * c_hi + hi * c_lo (mod 2^32), and the high word of
 // z ^ (z >> 31) is hi ^ (hi >> 31).
-__device__ __forceinline__ uint32_t splitmix64_hi32(uint64_t z) {
+// splitmix64_hi32 before its last xor-shift: u = h ^ (h >> 31), which differs
+// from h in bit 0 only, so the top 31 bits of u are those of h.
+__device__ __forceinline__ uint32_t splitmix64_hi32_pre(uint64_t z) {
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
     z ^= z >> 27;
     const uint32_t lo = (uint32_t)z, hi = (uint32_t)(z >> 32);
-    const uint32_t h = __umulhi(lo, 0x133111EBu) + lo * 0x94D049BBu + hi * 0x133111EBu;
+    return __umulhi(lo, 0x133111EBu) + lo * 0x94D049BBu + hi * 0x133111EBu;
+}
+__device__ __forceinline__ uint32_t splitmix64_hi32(uint64_t z) {
+    const uint32_t h = splitmix64_hi32_pre(z);
     return h ^ (h >> 31);
 }
 
@@ -330,9 +335,10 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
             uint32_t bits = 0, near = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t u = splitmix64_hi32(st + (uint64_t)i * kGamma);
-                const float x = __uint_as_float((u >> 9) | 0x3F800000u) - 1.0f;
-                const float s = fminf(fmaxf(f4_get(v, i), 0.f), 1.f);  // NaN -> 0
+                // u >> 9 (x' = u / 2^32 truncated to 23 bits) needs only the top bits
+                const uint32_t h = splitmix64_hi32_pre(st + (uint64_t)i * kGamma);
+                const float x = __uint_as_float((h >> 9) | 0x3F800000u) - 1.0f;
+                const float s = __saturatef(f4_get(v, i));  // clamped to [0, 1], NaN -> 0
                 const float d = __fmaf_rn(-s, K, x);
                 bits |= d < 0.f ? 1u << i : 0u;
                 near |= fabsf(d) <= margin ? 1u << i : 0u;

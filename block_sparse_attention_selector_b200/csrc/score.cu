@@ -16,10 +16,12 @@
 //       ranges minus log2(w) (+inf for an empty cluster);
 //   K3c absa_score_out_kernel      per (head, key range): the logits again,
 //       transposed (thread = key block), s = sum_c exp2(scaled logit - L_c).
-// Logits are mu_hi . (kbar_hi + kbar_lo) from two fp16 tcgen05 MMAs per
-// k-step; kbar is carried to about 2^-22 and mu to fp16 (relative rounding
-// 2^-12 on average), so a workload logit (|l| up to about 6 after scaling) is
-// off by about 1e-4 at most, an order below the 1e-3 score tolerance.
+// Logits of the score pass are mu_hi . (kbar_hi + kbar_lo) from two fp16
+// tcgen05 MMAs per k-step; kbar is carried to about 2^-22 and mu to fp16
+// (relative rounding 2^-12 on average), so a workload logit (|l| up to about
+// 6 after scaling) is off by about 1e-4 at most, an order below the 1e-3
+// score tolerance.  The log-sum-exp pass uses mu_hi . kbar_hi alone (see
+// ScoreCta::kLo).
 #include "absa_kernels.cuh"
 
 namespace absa {
@@ -56,6 +58,13 @@ struct Score2Smem {
 template <int D, bool TRANSPOSED>
 struct ScoreCta {
     using S = Score2Smem<D>;
+    // The log-sum-exp pass (not transposed) takes the logits mu_hi . kbar_hi
+    // alone: the dropped mu_hi . kbar_lo moves a scaled logit by about 1e-4
+    // (kbar_lo is the fp16 rounding remainder, 2^-11 of kbar), and the
+    // normaliser, a softmax-weighted average of exp over all key blocks,
+    // moves by the weighted mean of those shifts, well below the 1e-3 score
+    // tolerance.  The score pass needs each logit, so it keeps both products.
+    static constexpr bool kLo = TRANSPOSED;
     uint8_t *sm;
     uint64_t *key_full, *mu_full, *mu_empty, *d_full, *d_empty;
     uint32_t *tmem_slot;
@@ -109,18 +118,20 @@ struct ScoreCta {
                             const CUtensorMap *tm_mu_hi, int key_row0, int mu_row0, int nmt,
                             int32_t *status) {
         tma_prefetch_desc(tm_mu_hi);
-        mbar_arrive_expect_tx(key_full, kScoreKeyTiles * S::kKeyTileBytes);
+        mbar_arrive_expect_tx(key_full, kScoreKeyTiles * S::kKeyTileBytes / (kLo ? 1 : 2));
         const uint32_t kbase = smem_u32(sm + S::kKeyOff);
         for (int kt = 0; kt < kScoreKeyTiles; ++kt)
             for (int r = 0; r < S::kRegions; ++r) {
                 const uint32_t off = r * S::kKeyRegion + kt * S::kTile;
                 tma_load_2d(kbase + off, tm_kb_hi, 64 * r, key_row0 + 128 * kt, key_full);
-                tma_load_2d(kbase + S::kKeyLoOff + off, tm_kb_lo, 64 * r, key_row0 + 128 * kt,
-                            key_full);
+                if (kLo)
+                    tma_load_2d(kbase + S::kKeyLoOff + off, tm_kb_lo, 64 * r, key_row0 + 128 * kt,
+                                key_full);
             }
         for (int m = 0; m < nmt; ++m) {
             const int st = m & 1;
-            if (m >= 2 && !mbar_wait(mu_empty + st, ((m - 2) >> 1) & 1, status, abort_flag)) break;
+            if (m >= 2 && !mbar_wait(mu_empty + st, ((m - 2) >> 1) & 1, status, abort_flag, 0))
+                break;
             mbar_arrive_expect_tx(mu_full + st, S::kMuTileBytes);
             const uint32_t base = smem_u32(sm + S::kMuOff + st * S::kMuTileBytes);
             for (int r = 0; r < S::kRegions; ++r)
@@ -165,8 +176,9 @@ struct ScoreCta {
                     const uint32_t moff = (ks >> 2) * S::kTile + (ks & 3) * 32;
                     const uint64_t mu_d = sw128_desc(mu_base + moff, 16, 1024);
                     tc_mma_f16(dt, mu_d, sw128_desc(kbase + koff, 16, 1024), idesc256, ks > 0);
-                    tc_mma_f16(dt, mu_d, sw128_desc(kbase + S::kKeyLoOff + koff, 16, 1024),
-                               idesc256, 1);
+                    if (kLo)
+                        tc_mma_f16(dt, mu_d, sw128_desc(kbase + S::kKeyLoOff + koff, 16, 1024),
+                                   idesc256, 1);
                 }
             }
             tc_commit(d_full + buf);

@@ -22,7 +22,7 @@ def header_functions():
     with open(os.path.join(ROOT, "include", "absa.h")) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(absa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(absa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported(L):
