@@ -542,13 +542,16 @@ def run_sweep(args):
         a, b = a.float(), b.float()
         return float((a - b).norm() / b.norm())
 
+    def err_rms(a, b):
+        return float((a.float() - b.float()).pow(2).mean().sqrt())
+
     p0 = absa.params_for(w)
     for _ in range(2):
         o_dense, dense_ms = timed(lambda: absa.dense_reference(p0, q, k, v))
     dense_rms = float(o_dense.float().pow(2).mean().sqrt())
     v_rms = float(v.float().pow(2).mean().sqrt())
     for budget, design in [(b, d) for b in SWEEP_BUDGETS for d in ("poisson", "systematic")]:
-        sel, att, rel, blocks = [], [], [], []
+        sel, att, rel, err, blocks = [], [], [], [], []
         for seed in range(8):
             p = absa.params_for(w, seed=seed, budget=budget, sampling=design)
             (plan, _, _), t_sel = timed(lambda: absa.select_plan(p, q, k))
@@ -558,6 +561,7 @@ def run_sweep(args):
                 att.append(t_att)
             sel.append(t_sel)
             rel.append(rel_l2(o, o_dense))
+            err.append(err_rms(o, o_dense))
             blocks.append(float(plan.counts.float().mean()))
         line = {"kind": "density_sweep", "workload": w.name, "budget_blocks": budget,
                 "sampling": design,
@@ -567,7 +571,10 @@ def run_sweep(args):
                 "dense_ms": dense_ms, "rel_l2_vs_dense_mean_8_seeds": float(np.mean(rel)),
                 "rel_l2_vs_dense_std_8_seeds": float(np.std(rel)),
                 # v is N(0,1) noise, so the dense output (an average of many v rows) is small
-                # next to v; these two set the scale of the relative error above
+                # next to v, and the relative error above divides by that small number.  The
+                # error RMS in units of the value RMS does not, and falls with the budget as
+                # the Horvitz-Thompson variance does.
+                "err_rms_over_v_rms_mean_8_seeds": float(np.mean(err)) / v_rms,
                 "dense_output_rms": dense_rms, "v_rms": v_rms}
         print(json.dumps(line), flush=True)
 
