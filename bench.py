@@ -260,7 +260,7 @@ def measured_peaks():
 
 def recorded_traffic(kernel_src, w):
     """DRAM bytes per launch from the committed ncu summary, if it matches this source and
-    was taken on this layer (the 40-head Wan2.1 480p layer)."""
+    was taken on this layer with all of its heads (scaled from a capture of a few heads)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -269,10 +269,10 @@ def recorded_traffic(kernel_src, w):
     with open(kernel_src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()[:16]
     ent = rec.get("sparse_attention")
-    if ent and ent.get("source_sha256_16") == digest and ent.get("workload", w.name) == w.name \
-            and w.H == 40 and w.name.startswith("wan2.1_480p"):
-        return ent.get("dram_bytes_per_launch")
-    return None
+    full_heads = {"hunyuan_720p_33x45x80": 24, "wan2.1_480p_21x30x52": 40, "wan2.1_720p_21x45x80": 40}
+    if not ent or ent.get("source_sha256_16") != digest or full_heads.get(w.name) != w.H:
+        return None
+    return ent.get("dram_bytes_per_launch", {}).get(w.name)
 
 
 def selector_sampler_roofline(w, counts, kmeans_ms, score_ms, sample_ms, hbm_gbs, peak_src):
