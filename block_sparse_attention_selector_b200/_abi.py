@@ -29,6 +29,7 @@ EXPORTED = (
     "absa_sparse_attention", "absa_dense_reference", "absa_plan_check",
     "absa_select_scores_static", "absa_step_host", "absa_select_pool_kmeans",
     "absa_select_block_scores", "absa_select_check", "absa_selftest_wait_timeout",
+    "absa_sparse_attention_pairs",
 )
 
 ABSA_STATIC_SCRATCH_BYTES = 64 << 20
@@ -95,6 +96,9 @@ def lib():
         L.absa_select_plan.restype = st
         L.absa_sparse_attention.argtypes = [P, vp, vp, vp, Q, vp, vp]
         L.absa_sparse_attention.restype = st
+        if hasattr(L, "absa_sparse_attention_pairs"):
+            L.absa_sparse_attention_pairs.argtypes = [P, vp, vp, vp, Q, vp, vp]
+            L.absa_sparse_attention_pairs.restype = st
         L.absa_dense_reference.argtypes = [P, vp, vp, vp, vp, vp, vp]
         L.absa_dense_reference.restype = st
         L.absa_plan_check.argtypes = [Q, vp]
@@ -157,6 +161,11 @@ def absa_select_plan(p, q, k, scores, plan, ws, ws_bytes, stream):
 
 def absa_sparse_attention(p, q, k, v, plan, o, stream):
     return lib().absa_sparse_attention(ctypes.byref(p), q, k, v, ctypes.byref(plan), o, stream)
+
+
+def absa_sparse_attention_pairs(p, q, k, v, plan, o, stream):
+    return lib().absa_sparse_attention_pairs(ctypes.byref(p), q, k, v, ctypes.byref(plan), o,
+                                             stream)
 
 
 def absa_dense_reference(p, q, k, v, o, status, stream):

@@ -310,6 +310,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// a += the bf16 in the low half of pk, b += the bf16 in the high half (each
+// widened exactly, then one f32 add: mixed-precision add of sm_100)
+__device__ __forceinline__ void add_bf16x2_f32(uint32_t pk, float &a, float &b) {
+    asm("{.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;}"
+        : "+f"(a), "+f"(b)
+        : "r"(pk));
+}
+
 // SplitMix64 output function (Steele, Lea and Flood, OOPSLA 2014).
 __device__ __forceinline__ uint64_t splitmix64_mix(uint64_t z) {
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;

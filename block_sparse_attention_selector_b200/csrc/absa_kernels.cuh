@@ -50,4 +50,15 @@ cudaError_t launch_attention(bool dense, const CUtensorMap &tq, const CUtensorMa
                              const int32_t *kv_index, const float *log_pi, int cap,
                              int32_t *status, cudaStream_t stream);
 
+// K5 under the paired design: one CTA per pair of query blocks (2p, 2p+1) of
+// a head, gathering the union of the two plan rows once.  The union list is
+// held in shared memory, so the host uses it only for 2 * cap <= kPairUnionMax.
+constexpr int kPairUnionMax = 6144;
+cudaError_t launch_attention_pair(const CUtensorMap &tq, const CUtensorMap &tk,
+                                  const CUtensorMap &tv, __nv_bfloat16 *o, int64_t BH, int N,
+                                  int nqb, int nkb, int d, float softmax_scale,
+                                  const int32_t *counts, const int32_t *kv_index,
+                                  const float *log_pi, int cap, int32_t *status,
+                                  cudaStream_t stream);
+
 }  // namespace absa

@@ -304,7 +304,7 @@ absa_status sample_plan_run(const absa_params *p, const float *scores, const abs
 
 absa_status attention_run(const absa_params *p, const void *q, const void *k, const void *v,
                           const absa_plan *plan, void *o, int32_t *status, HeadRun hr,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool pairs = false) {
     const Dims dm = dims_of(p);
     const int64_t off = hr.bh0 * p->N * (int64_t)p->d;
     const auto *qh = static_cast<const __nv_bfloat16 *>(q) + off;
@@ -324,6 +324,12 @@ absa_status attention_run(const absa_params *p, const void *q, const void *k, co
                                           dm.nkb, p->d, p->softmax_scale, nullptr, nullptr,
                                           nullptr, 0, status, s));
     const int64_t row0 = hr.bh0 * dm.nqb, cap = plan->capacity;
+    if (pairs)
+        return from_cuda(launch_attention_pair(tq, tk, tv, oh, hr.nbh, p->N, dm.nqb, dm.nkb,
+                                               p->d, p->softmax_scale, plan->counts + row0,
+                                               plan->kv_index + row0 * cap,
+                                               plan->log_pi + row0 * cap, plan->capacity,
+                                               plan->status, s));
     return from_cuda(launch_attention(false, tq, tk, tv, kh, vh, oh, hr.nbh, p->N, dm.nqb,
                                       dm.nkb, p->d, p->softmax_scale, plan->counts + row0,
                                       plan->kv_index + row0 * cap, plan->log_pi + row0 * cap,
@@ -494,6 +500,22 @@ absa_status absa_sparse_attention(const absa_params *p, const void *q, const voi
         return ABSA_ERR_INVALID_ARG;
     return attention_run(p, q, k, v, plan, o, plan->status, all_heads(p),
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+absa_status absa_sparse_attention_pairs(const absa_params *p, const void *q, const void *k,
+                                        const void *v, const absa_plan *plan, void *o,
+                                        void *stream) {
+    NvtxRange range("absa_sparse_attention_pairs");
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    st = check_plan(p, plan);
+    if (st != ABSA_OK) return st;
+    if (!q || !k || !v || !o) return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return ABSA_ERR_INVALID_ARG;
+    if (2 * (int64_t)plan->capacity > kPairUnionMax) return ABSA_ERR_UNSUPPORTED;
+    return attention_run(p, q, k, v, plan, o, plan->status, all_heads(p),
+                         reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,

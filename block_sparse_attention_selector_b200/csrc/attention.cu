@@ -23,7 +23,9 @@
 // Softmax works in the exp2 domain: x = log2(e) * scale * (q.k) + bias with
 // bias = -log2(pi) for a valid token and -inf for padding; the row maximum is
 // updated lazily (O is rescaled only when the max grows by more than 2^8), and
-// the final O is divided by the fp32 row sum.
+// the final O is divided by the fp32 sum of the bf16-rounded P, the weights
+// the PV product used (a row dominated by a few tokens then returns their
+// values without the rounding of P showing).
 #include "absa_kernels.cuh"
 
 namespace absa {
@@ -415,7 +417,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             m_ref = m_new;
             const float moff = m_ref == -INFINITY ? 0.f : -m_ref;
             const uint64_t moff2 = ((uint64_t)__float_as_uint(moff) << 32) | __float_as_uint(moff);
-            uint64_t acc2[4] = {0, 0, 0, 0};
+            // row sum of the bf16-rounded P: the weights the PV product uses
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {  // P_j in two halves of 16 columns (32 keys)
                 uint32_t pk[16];
@@ -425,18 +428,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                         f32x2_add(((uint64_t)sv[ch][e + 1] << 32) | sv[ch][e], moff2);
                     const float p0 = ex2(__uint_as_float((uint32_t)y2));
                     const float p1 = ex2(__uint_as_float((uint32_t)(y2 >> 32)));
-                    acc2[(e >> 1) & 3] = f32x2_add(acc2[(e >> 1) & 3],
-                                                   ((uint64_t)__float_as_uint(p1) << 32) | __float_as_uint(p0));
                     pk[e >> 1] = pack_bf16x2(p0, p1);
+                    add_bf16x2_f32(pk[e >> 1], acc[2 * ((e >> 1) & 1)], acc[2 * ((e >> 1) & 1) + 1]);
                 }
                 tmem_st16(s_t + 16 * ch, pk);
             }
-            float tsum;
-            {
-                const uint64_t a01 = f32x2_add(acc2[0], acc2[1]), a23 = f32x2_add(acc2[2], acc2[3]);
-                const uint64_t a = f32x2_add(a01, a23);
-                tsum = __uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)(a >> 32));
-            }
+            const float tsum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             if (any_need) {  // lazy rescale of O by exp2(m_old - m_new) once PV_{j-1} is done
                 ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1,
                                                        status, abort_flag));

@@ -220,6 +220,24 @@ absa_status absa_select_plan(const absa_params *p, const void *q, const void *k,
 absa_status absa_sparse_attention(const absa_params *p, const void *q, const void *k,
                                   const void *v, const absa_plan *plan, void *o, void *stream);
 
+/* absa_sparse_attention computed with one CTA per pair of query blocks
+ * (2p, 2p+1) of a head (SIP paragraph, with the paired design of
+ * absa_sample_plan): the CTA gathers each key/value block of the union of the
+ * two plan rows once and runs one softmax chain per query block over it, a
+ * block absent from a row entering that row's chain with logit bias -inf.
+ * Any plan is accepted (rows out of order or with repeated ids are processed
+ * as the concatenation of the two rows), and every row's output is the
+ * absa_sparse_attention output up to summation order; bad rows are rejected
+ * as there.  The union list lives in shared memory: plan->capacity must be
+ * at most 3072 (ABSA_ERR_UNSUPPORTED otherwise).  The paired design makes
+ * the union only 10-18% larger than one row, yet on B200 this form measured
+ * slower than absa_sparse_attention (two independent single-block CTAs per
+ * SM), which the other entry points use; it is kept as the pair-union
+ * variant of the attention. */
+absa_status absa_sparse_attention_pairs(const absa_params *p, const void *q, const void *k,
+                                        const void *v, const absa_plan *plan, void *o,
+                                        void *stream);
+
 /* Dense softmax attention (the full-attention reference of the pages'
  * evaluation) with the same tile machinery over contiguous keys.  status is
  * a device word for ABSA_DEVFLAG_TIMEOUT (may be NULL). */

@@ -105,6 +105,14 @@ def test_entry_points_reject_null_and_misaligned_pointers_before_cuda(L):
     bad = _abi.absa_plan(5, 128, 96, 16, 16, 16, 16, 16)
     assert _abi.absa_sparse_attention(p, 16, 16, 16, bad, 16, None) == _abi.ABSA_ERR_INVALID_ARG
     assert _abi.absa_plan_check(_abi.absa_plan(), None) == _abi.ABSA_ERR_INVALID_ARG
+    # the pair-union attention: same checks, and a capacity above its union list
+    pairs = _abi.absa_sparse_attention_pairs
+    assert pairs(p, 16, 16, 16, plan, 16, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert pairs(p, 16, 16, 16, bad, 16, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert pairs(p, 16, 16, 8, _abi.absa_plan(4, 128, 96, 16, 16, 16, 16, 16), 16,
+                 None) == _abi.ABSA_ERR_INVALID_ARG
+    wide = _abi.absa_plan(4, 128, 3073, 16, 16, 16, 16, 16)
+    assert pairs(p, 16, 16, 16, wide, 16, None) == _abi.ABSA_ERR_UNSUPPORTED
     # the host-buffer step: null host pointers, an empty head run, a short workspace
     good = _abi.absa_plan(4, 128, 96, 16, 16, 16, 16, 16)
     step = _abi.absa_step_host
