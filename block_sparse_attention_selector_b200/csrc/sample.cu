@@ -17,12 +17,13 @@
 
 namespace absa {
 
-// q - 1 as a u32 (q = max(1, floor(s 2^32)) <= 2^32).
+// q - 1 as a u32 (q = max(1, floor(s 2^32)) <= 2^32).  The truncating
+// conversion saturates (NaN and negatives give 0, x >= 2^32 gives 2^32 - 1,
+// and no float lies in (2^32 - 256, 2^32)), so f = floor(x) clamped; then
+// q - 1 = f - 1 except for f = 0 (q = 1) and the saturated f (q = 2^32).
 __device__ __forceinline__ uint32_t quantise_m1(float s) {
-    const float x = s * 4294967296.0f;  // exact power-of-two scaling
-    if (!(x >= 1.0f)) return 0u;        // NaN, negative, or below one unit
-    if (x >= 4294967296.0f) return 0xFFFFFFFFu;
-    return __float2uint_rz(x) - 1u;     // floor for 1 <= x < 2^32
+    const uint32_t f = __float2uint_rz(s * 4294967296.0f);  // exact power-of-two scaling
+    return f - ((f - 1u) < 0xFFFFFFFEu ? 1u : 0u);
 }
 
 constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;  // SplitMix64 increment
@@ -100,12 +101,16 @@ struct ScoreRow {
     const float *s;
     const float4 *s4;
     int nkb, off, nchunks;
+    int full0, full1;  // chunks [full0, full1) hold 4 blocks of the row each
 
     __device__ ScoreRow(const float *row, int nkb_) : s(row), nkb(nkb_) {
         off = (int)((reinterpret_cast<uintptr_t>(row) >> 2) & 3u);
         s4 = reinterpret_cast<const float4 *>(row - off);
         nchunks = (nkb + off + 3) >> 2;
+        full0 = off ? 1 : 0;
+        full1 = (nkb + off) >> 2;
     }
+    __device__ bool full(int c) const { return c >= full0 && c < full1; }
     __device__ float4 chunk(int c) const {
         const int j0 = 4 * c - off;
         if (c >= nchunks) return make_float4(0.f, 0.f, 0.f, 0.f);
@@ -126,6 +131,14 @@ struct ScoreRow {
         return m;
     }
 };
+
+// The low 8 bits of x moved to bits 0, 4, 8, ..., 28.
+__device__ __forceinline__ uint32_t spread8(uint32_t x) {
+    x &= 0xFFu;
+    x = (x | (x << 12)) & 0x000F000Fu;
+    x = (x | (x << 6)) & 0x03030303u;
+    return (x | (x << 3)) & 0x11111111u;
+}
 
 __device__ __forceinline__ float f4_get(const float4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
@@ -217,26 +230,40 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
     uint64_t R0 = 0;
     {
         constexpr int kAhead = 4;  // tiles in flight per thread
+        uint64_t qsum = 0;             // sum of q - 1 over the valid blocks
+        int nvalid = 0;
         for (int t0 = 0; t0 < ntiles; t0 += kAhead) {
             float4 v[kAhead];
 #pragma unroll
-            for (int u = 0; u < kAhead; ++u) v[u] = sr.chunk((t0 + u) * kThreads + tid);
+            for (int u = 0; u < kAhead; ++u) {
+                const int c = (t0 + u) * kThreads + tid;
+                v[u] = sr.full(c) ? __ldg(sr.s4 + c) : sr.chunk(c);
+            }
 #pragma unroll
             for (int u = 0; u < kAhead; ++u) {
                 const int c = (t0 + u) * kThreads + tid;
-                const uint32_t valid = sr.valid_mask(c);
-                uint32_t qm[4];
-                int nc = 0;
+                const uint32_t q0 = quantise_m1(v[u].x), q1 = quantise_m1(v[u].y);
+                const uint32_t q2 = quantise_m1(v[u].z), q3 = quantise_m1(v[u].w);
+                uint32_t qm[4] = {q0, q1, q2, q3};
+                uint32_t valid = 0xFu;
+                if (sr.full(c)) {  // the common case: no mask
+                    qsum += ((uint64_t)q0 + q1) + ((uint64_t)q2 + q3);
+                    nvalid += 4;
+                } else {
+                    valid = sr.valid_mask(c);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    qm[i] = quantise_m1(f4_get(v[u], i));
-                    if ((valid >> i) & 1u) {
-                        R0 += (uint64_t)qm[i] + 1;
-                        nc += qm[i] >= t_list_m1 ? 1 : 0;
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        if ((valid >> i) & 1u) {
+                            qsum += qm[i];
+                            ++nvalid;
+                        }
                 }
-                if (nc) {  // rare: append this thread's listed blocks
-                    int p = atomicAdd(&n_cand, nc);
+                // rare: a listed block in this chunk
+                if (max(max(q0, q1), max(q2, q3)) >= t_list_m1) {
+                    int nc = 0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) nc += ((valid >> i) & 1u) && qm[i] >= t_list_m1;
+                    int p = nc ? atomicAdd(&n_cand, nc) : 0;
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         if (((valid >> i) & 1u) && qm[i] >= t_list_m1) {
@@ -246,6 +273,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
                 }
             }
         }
+        R0 = qsum + (uint64_t)nvalid;
     }
     int dummy = 0;
     block_sum2<WARPS>(R0, dummy, red_a, red_b);  // its barriers also publish n_cand and cand
@@ -302,7 +330,6 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
     const int niters = (sr.nchunks + 31) >> 5;
     const int per = (niters + WARPS - 1) / WARPS;
     const int i0 = min(niters, warp * per), i1 = min(niters, i0 + per);
-    const uint32_t below = (1u << lane) - 1u;
     int wtaken = 0;  // taken blocks of this warp's segment
     // exact take bits of the 4 blocks of chunk c (capped, or the exact draw)
     auto exact_bits = [&](const float4 &v, uint64_t st, uint32_t which) -> uint32_t {
@@ -330,22 +357,34 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
         uint64_t st = base + (uint64_t)(int64_t)(4 * (i0 * 32 + lane) - sr.off) * kGamma;
         for (int it = i0; it < i1; ++it, st += 128 * kGamma) {
             const int c = it * 32 + lane;
-            const float4 v = sr.chunk(c);
-            const uint32_t valid = sr.valid_mask(c);
-            uint32_t bits = 0, near = 0;
+            const bool full = sr.full(c);
+            const float4 v = full ? __ldg(sr.s4 + c) : sr.chunk(c);
+            uint32_t bits = 0;
+            float dmin = INFINITY;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                // u >> 9 (x' = u / 2^32 truncated to 23 bits) needs only the top bits
+                // x' = 1 + u / 2^32 truncated to 23 bits needs only the top bits
+                // of u; taken iff x' - s' K < 1
                 const uint32_t h = splitmix64_hi32_pre(st + (uint64_t)i * kGamma);
-                const float x = __uint_as_float((h >> 9) | 0x3F800000u) - 1.0f;
-                const float s = __saturatef(f4_get(v, i));  // clamped to [0, 1], NaN -> 0
-                const float d = __fmaf_rn(-s, K, x);
-                bits |= d < 0.f ? 1u << i : 0u;
-                near |= fabsf(d) <= margin ? 1u << i : 0u;
+                const float x1 = __uint_as_float((h >> 9) | 0x3F800000u);
+                const float sc = __saturatef(f4_get(v, i));  // clamped to [0, 1], NaN -> 0
+                const float d1 = __fmaf_rn(-sc, K, x1);
+                bits |= d1 < 1.0f ? 1u << i : 0u;
+                dmin = fminf(dmin, fabsf(d1 - 1.0f));
             }
-            near &= valid;
-            if (__any_sync(0xffffffffu, near != 0))  // rare: exact test near the threshold
+            const uint32_t valid = full ? 0xFu : sr.valid_mask(c);
+            if (__any_sync(0xffffffffu, dmin <= margin)) {  // rare: exact test near the threshold
+                uint32_t near = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t h = splitmix64_hi32_pre(st + (uint64_t)i * kGamma);
+                    const float x1 = __uint_as_float((h >> 9) | 0x3F800000u);
+                    const float d1 = __fmaf_rn(-__saturatef(f4_get(v, i)), K, x1);
+                    near |= fabsf(d1 - 1.0f) <= margin ? 1u << i : 0u;
+                }
+                near &= valid;
                 bits = (bits & ~near) | exact_bits(v, st, near);
+            }
             store_bits(it, bits & valid);
         }
     } else {
@@ -422,29 +461,52 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 6 : 3) absa_sample_ke
         pos += w < warp ? x : 0;
         total += x;
     }
-    for (int it = i0; it < i1 && pos < cap; ++it) {
-        const uint4 W = takew[it];
-        const uint32_t nib = ((W.x >> lane) & 1u) | (((W.y >> lane) & 1u) << 1) |
-                             (((W.z >> lane) & 1u) << 2) | (((W.w >> lane) & 1u) << 3);
-        int p = pos + __popc(W.x & below) + __popc(W.y & below) + __popc(W.z & below) +
-                __popc(W.w & below);
-        const int j0 = 4 * (it * 32 + lane) - sr.off;
+    // Lane l takes 32 consecutive blocks at a time: block-order word l % 4 of
+    // step l / 4 of a group of 8 steps, interleaved from the step's 4 ballots
+    // (bit 4m + i of word k is take bit i of lane 8k + m); one warp scan of
+    // the words' counts places them.
+    for (int g0 = i0; g0 < i1 && pos < cap; g0 += 8) {
+        const int it = g0 + (lane >> 2), k8 = 8 * (lane & 3);
+        uint32_t word = 0;
+        if (it < i1) {
+            const uint4 W = takew[it];
+            word = spread8(W.x >> k8) | (spread8(W.y >> k8) << 1) | (spread8(W.z >> k8) << 2) |
+                   (spread8(W.w >> k8) << 3);
+        }
+        const int cnt = __popc(word);
+        int inc = cnt;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if ((nib >> i) & 1u) {
-                if (p < cap) idx_row[p] = j0 + i;
-                ++p;
-            }
-        pos += __popc(W.x) + __popc(W.y) + __popc(W.z) + __popc(W.w);
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        int p = pos + inc - cnt;
+        const int jb = 128 * it + 4 * k8 - sr.off;
+        while (word) {
+            const int b = __ffs(word) - 1;
+            word &= word - 1;
+            if (p < cap) idx_row[p] = jb + b;
+            ++p;
+        }
+        pos += __shfl_sync(0xffffffffu, inc, 31);
     }
     __syncthreads();  // the kv_index entries written above are visible to the whole CTA
 
     // ---- ln(pi) of the written entries
     const int written = min(total, cap);
-    for (int p = tid; p < written; p += kThreads) {
-        const uint32_t qmp = quantise_m1(__ldg(srow + idx_row[p]));
-        const uint64_t rqp = (uint64_t)r32 * qmp + r32;
-        lp_row[p] = rqp >= R ? 0.f : (float)log((double)rqp / (double)R);
+    for (int p0 = tid; p0 < written; p0 += 4 * kThreads) {  // 4 entries in flight per thread
+        int id[4];
+        float sv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) id[u] = p0 + u * kThreads < written ? idx_row[p0 + u * kThreads] : 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) sv[u] = __ldg(srow + id[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int p = p0 + u * kThreads;
+            const uint64_t rqp = (uint64_t)r32 * quantise_m1(sv[u]) + r32;
+            if (p < written) lp_row[p] = rqp >= R ? 0.f : (float)log((double)rqp / (double)R);
+        }
     }
     if (tid == 0) {
         counts[row] = written;
