@@ -48,6 +48,8 @@ def lib():
         L.oracle_sparse_attention_rows.argtypes = [_u16p, _i32, _i32, _u16p, _u16p, _i64, _i32p,
                                                    _f32p, _i32, _dbl, _f64p]
         L.oracle_dense_attention_rows.argtypes = [_u16p, _i32, _i32, _u16p, _u16p, _i64, _dbl, _f64p]
+        L.oracle_remainder_attention_rows.argtypes = [_u16p, _i32, _i32, _u16p, _u16p, _i64, _i32p,
+                                                      _i32, _i32, _dbl, _f64p]
         L.oracle_ht_parts.argtypes = [_u16p, _i32, _u16p, _u16p, _i64, _i32p, _f32p, _i32, _dbl,
                                       _dbl, _f64p, ctypes.POINTER(_dbl)]
         L.oracle_select_scores.argtypes = [_i32, _i32, _i64, _i32, _i32, _i32, _dbl, _u16p, _u16p,
@@ -170,6 +172,48 @@ def sparse_attention_rows(q, k, v, blocks, log_pi, scale):
     o = np.empty((m, d), np.float64)
     lib().oracle_sparse_attention_rows(q, m, d, k, v, k.shape[0], blocks, log_pi, blocks.shape[0],
                                        float(scale), o)
+    return o
+
+
+REMAINDER_GROUP_BLOCKS = 32  # key blocks per remainder group (128 tokens)
+
+
+def remainder_attention_rows(q, k, v, blocks, scale, group_blocks=REMAINDER_GROUP_BLOCKS):
+    """ESTRA-style attention of query rows q [m,d]: the listed blocks exactly,
+    the rest of every group of `group_blocks` key blocks through its
+    variance-corrected representative (fp64 out)."""
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    blocks = _c(blocks, np.int32)
+    m, d = q.shape
+    o = np.empty((m, d), np.float64)
+    lib().oracle_remainder_attention_rows(q, m, d, k, v, k.shape[0], blocks, blocks.shape[0],
+                                          int(group_blocks), float(scale), o)
+    return o
+
+
+def remainder_attention(q, k, v, plan, scale=None, qb_range=(0, 0),
+                        group_blocks=REMAINDER_GROUP_BLOCKS):
+    """ESTRA-style attention over a whole layer with the plan's blocks as the
+    exact part (fp64 [B,H,N,d]; rows outside qb_range are NaN)."""
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    counts, idx = plan["counts"], plan["kv_index"]
+    nqb = idx.shape[2]
+    lo, hi = qb_range if qb_range != (0, 0) else (0, nqb)
+    o = np.full((B, H, N, d), np.nan, np.float64)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(lo, hi):
+                rows = slice(128 * qb, min(N, 128 * qb + 128))
+                c = int(counts[b, h, qb])
+                o[b, h, rows] = remainder_attention_rows(q[b, h, rows], k[b, h], v[b, h],
+                                                         idx[b, h, qb, :c], scale, group_blocks)
     return o
 
 

@@ -377,6 +377,135 @@ void oracle_sparse_attention_rows(const uint16_t *q, int nrows, int d,
     free(num);
 }
 
+/* ESTRA-style remainder (ESTRA page, summary and figure: cluster, compute the
+ * selected pairs exactly, approximate the rest from group averages with a
+ * variance-calibrated mean correction).  Reading: the listed blocks are the
+ * exact part (no ln pi shift); the keys are grouped into runs of
+ * `group_blocks` consecutive 4-token blocks; every group g contributes one
+ * representative with the mean key mu_g and mean value nu_g of its tokens,
+ * weight m_g = tokens of g not in the listed blocks, and the correction of
+ * the mean for the spread of the keys taken as isotropic:
+ *   sum_{t in rest of g} exp(s q.k_t) ~ m_g exp(s q.mu_g + s^2 |q|^2 var_g / 2),
+ * var_g = (1/d) sum_e (mean_t k_te^2 - mu_ge^2)  (the identity
+ * E exp(X) = exp(E X + Var X / 2) of a Gaussian X = s q.k).  One softmax
+ * runs over the exact tokens and the representatives together. */
+void oracle_remainder_attention_rows(const uint16_t *q, int nrows, int d,
+                                     const uint16_t *k, const uint16_t *v,
+                                     int64_t N, const int32_t *blocks, int count,
+                                     int group_blocks, double scale, double *o)
+{
+    const int64_t nkb = (N + 3) / 4;
+    const int64_t ng = (nkb + group_blocks - 1) / group_blocks;
+    double *mu = (double *)calloc((size_t)(ng * d), sizeof(double));
+    double *nu = (double *)calloc((size_t)(ng * d), sizeof(double));
+    double *var = (double *)calloc((size_t)ng, sizeof(double));
+    double *rest = (double *)calloc((size_t)ng, sizeof(double));
+    double *sq = (double *)malloc(sizeof(double) * (size_t)d);
+    /* group statistics over all tokens of each group */
+    for (int64_t g = 0; g < ng; ++g) {
+        const int64_t t0 = 4 * g * group_blocks;
+        int64_t t1 = t0 + 4 * (int64_t)group_blocks;
+        if (t1 > N)
+            t1 = N;
+        const double n = (double)(t1 - t0);
+        for (int e = 0; e < d; ++e)
+            sq[e] = 0.0;
+        for (int64_t t = t0; t < t1; ++t)
+            for (int e = 0; e < d; ++e) {
+                const double kv = (double)oracle_bf16_to_float(k[t * d + e]);
+                mu[g * d + e] += kv;
+                sq[e] += kv * kv;
+                nu[g * d + e] += (double)oracle_bf16_to_float(v[t * d + e]);
+            }
+        double vs = 0.0;
+        for (int e = 0; e < d; ++e) {
+            mu[g * d + e] /= n;
+            nu[g * d + e] /= n;
+            double ve = sq[e] / n - mu[g * d + e] * mu[g * d + e];
+            vs += ve > 0.0 ? ve : 0.0;
+        }
+        var[g] = vs / (double)d;
+        rest[g] = n;
+    }
+    /* tokens of the listed blocks leave their group's rest */
+    for (int b = 0; b < count; ++b) {
+        const int64_t j = blocks[b];
+        if (j < 0 || j >= nkb)
+            continue;
+        int64_t ntok = N - 4 * j;
+        if (ntok > 4)
+            ntok = 4;
+        rest[j / group_blocks] -= (double)ntok;
+    }
+    const int64_t ntok_exact = 4 * (int64_t)(count > 0 ? count : 1);
+    double *l = (double *)malloc(sizeof(double) * (size_t)(ntok_exact + ng));
+    int64_t *tok = (int64_t *)malloc(sizeof(int64_t) * (size_t)ntok_exact);
+    float *qf = (float *)malloc(sizeof(float) * (size_t)d);
+    for (int r = 0; r < nrows; ++r) {
+        double qq = 0.0;
+        for (int e = 0; e < d; ++e) {
+            qf[e] = oracle_bf16_to_float(q[(size_t)r * d + e]);
+            qq += (double)qf[e] * (double)qf[e];
+        }
+        double mx = -INFINITY;
+        int64_t p = 0;
+        for (int b = 0; b < count; ++b)
+            for (int t = 0; t < 4; ++t) {
+                const int64_t n = 4 * (int64_t)blocks[b] + t;
+                if (blocks[b] < 0 || n >= N)
+                    continue;
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e)
+                    dot += (double)qf[e] * (double)oracle_bf16_to_float(k[n * d + e]);
+                l[p] = scale * dot;
+                tok[p] = n;
+                if (l[p] > mx)
+                    mx = l[p];
+                p += 1;
+            }
+        for (int64_t g = 0; g < ng; ++g) {
+            double *lg = &l[p + g];
+            if (rest[g] <= 0.0) {
+                *lg = -INFINITY;
+                continue;
+            }
+            double dot = 0.0;
+            for (int e = 0; e < d; ++e)
+                dot += (double)qf[e] * mu[g * d + e];
+            *lg = scale * dot + 0.5 * scale * scale * qq * var[g] + log(rest[g]);
+            if (*lg > mx)
+                mx = *lg;
+        }
+        double den = 0.0;
+        for (int e = 0; e < d; ++e)
+            o[(size_t)r * d + e] = 0.0;
+        for (int64_t i = 0; i < p; ++i) {
+            const double w = exp(l[i] - mx);
+            den += w;
+            for (int e = 0; e < d; ++e)
+                o[(size_t)r * d + e] += w * (double)oracle_bf16_to_float(v[tok[i] * d + e]);
+        }
+        for (int64_t g = 0; g < ng; ++g) {
+            if (l[p + g] == -INFINITY)
+                continue;
+            const double w = exp(l[p + g] - mx);
+            den += w;
+            for (int e = 0; e < d; ++e)
+                o[(size_t)r * d + e] += w * nu[g * d + e];
+        }
+        for (int e = 0; e < d; ++e)
+            o[(size_t)r * d + e] = den > 0.0 ? o[(size_t)r * d + e] / den : 0.0;
+    }
+    free(mu);
+    free(nu);
+    free(var);
+    free(rest);
+    free(sq);
+    free(l);
+    free(tok);
+    free(qf);
+}
+
 void oracle_dense_attention_rows(const uint16_t *q, int nrows, int d,
                                  const uint16_t *k, const uint16_t *v,
                                  int64_t N, double scale, double *o)

@@ -124,6 +124,17 @@ void oracle_sparse_attention_rows(const uint16_t *q, int nrows, int d,
 
 /* Dense softmax attention for `nrows` query rows over all N tokens of the
  * head: the full-attention reference of the evaluation section.  fp64. */
+/* ESTRA-style remainder attention of query rows q [nrows,d] of one head:
+ * the listed blocks exactly (no ln pi shift), every group of group_blocks
+ * consecutive 4-token blocks as one representative (mean key, mean value,
+ * weight = its tokens outside the listed blocks, log-weight corrected by
+ * s^2 |q|^2 var_g / 2 with var_g the per-dimension key variance averaged
+ * over dimensions); one softmax over both.  o is fp64 [nrows,d]. */
+void oracle_remainder_attention_rows(const uint16_t *q, int nrows, int d,
+                                     const uint16_t *k, const uint16_t *v,
+                                     int64_t N, const int32_t *blocks, int count,
+                                     int group_blocks, double scale, double *o);
+
 void oracle_dense_attention_rows(const uint16_t *q, int nrows, int d,
                                  const uint16_t *k, const uint16_t *v,
                                  int64_t N, double scale, double *o);
