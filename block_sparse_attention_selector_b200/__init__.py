@@ -14,6 +14,7 @@ from ._abi import (AbsaError, absa_check_params, absa_dense_reference, absa_para
                    absa_plan_capacity, absa_plan_check, absa_sample_plan,
                    absa_select_block_scores, absa_select_check, absa_select_plan,
                    absa_select_pool_kmeans, absa_select_scores, absa_sparse_attention,
+                   absa_remainder_attention, absa_remainder_workspace_bytes,
                    absa_sparse_attention_pairs, absa_step_host, absa_workspace_bytes)
 from .synthetic import Workload
 
@@ -21,10 +22,12 @@ __all__ = [
     "AbsaError", "Plan", "Workload", "absa_check_params", "absa_dense_reference", "absa_params",
     "absa_plan", "absa_plan_capacity", "absa_plan_check", "absa_sample_plan", "absa_select_plan",
     "absa_select_block_scores", "absa_select_check", "absa_select_pool_kmeans",
-    "absa_select_scores", "absa_sparse_attention", "absa_sparse_attention_pairs", "absa_step_host",
+    "absa_remainder_attention", "absa_remainder_workspace_bytes", "absa_select_scores",
+    "absa_sparse_attention", "absa_sparse_attention_pairs", "absa_step_host",
     "absa_workspace_bytes",
     "block_scores", "dense_reference", "make_params", "pool_kmeans", "sample_plan", "select_check",
-    "select_plan", "select_scores", "sparse_attention", "sparse_attention_pairs", "step_host",
+    "remainder_attention", "select_plan", "select_scores", "sparse_attention",
+    "sparse_attention_pairs", "step_host",
     "workspace", "version",
 ]
 
@@ -197,6 +200,23 @@ def sparse_attention_pairs(p, q, k, v, plan, out=None, stream=None):
         out = torch.empty_like(q)
     _abi.check(absa_sparse_attention_pairs(p, _ptr(q), _ptr(k), _ptr(v), plan.c, _ptr(out),
                                            _stream_handle(stream)), "absa_sparse_attention_pairs")
+    return out
+
+
+def remainder_attention(p, q, k, v, plan, out=None, ws=None, stream=None):
+    """ESTRA-style attention: the plan's blocks exact, every group of 32 key
+    blocks through its variance-corrected representative (include/absa.h)."""
+    import torch
+
+    _check_bf16(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    nbytes = absa_remainder_workspace_bytes(p)
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _abi.check(absa_remainder_attention(p, _ptr(q), _ptr(k), _ptr(v), plan.c, _ptr(out), _ptr(ws),
+                                        ws.numel(), _stream_handle(stream)),
+               "absa_remainder_attention")
     return out
 
 

@@ -29,7 +29,7 @@ EXPORTED = (
     "absa_sparse_attention", "absa_dense_reference", "absa_plan_check",
     "absa_select_scores_static", "absa_step_host", "absa_select_pool_kmeans",
     "absa_select_block_scores", "absa_select_check", "absa_selftest_wait_timeout",
-    "absa_sparse_attention_pairs",
+    "absa_sparse_attention_pairs", "absa_remainder_workspace_bytes", "absa_remainder_attention",
 )
 
 ABSA_STATIC_SCRATCH_BYTES = 64 << 20
@@ -96,6 +96,11 @@ def lib():
         L.absa_select_plan.restype = st
         L.absa_sparse_attention.argtypes = [P, vp, vp, vp, Q, vp, vp]
         L.absa_sparse_attention.restype = st
+        if hasattr(L, "absa_remainder_attention"):
+            L.absa_remainder_workspace_bytes.argtypes = [P]
+            L.absa_remainder_workspace_bytes.restype = ctypes.c_size_t
+            L.absa_remainder_attention.argtypes = [P, vp, vp, vp, Q, vp, vp, ctypes.c_size_t, vp]
+            L.absa_remainder_attention.restype = st
         if hasattr(L, "absa_sparse_attention_pairs"):
             L.absa_sparse_attention_pairs.argtypes = [P, vp, vp, vp, Q, vp, vp]
             L.absa_sparse_attention_pairs.restype = st
@@ -166,6 +171,15 @@ def absa_sparse_attention(p, q, k, v, plan, o, stream):
 def absa_sparse_attention_pairs(p, q, k, v, plan, o, stream):
     return lib().absa_sparse_attention_pairs(ctypes.byref(p), q, k, v, ctypes.byref(plan), o,
                                              stream)
+
+
+def absa_remainder_workspace_bytes(p):
+    return lib().absa_remainder_workspace_bytes(ctypes.byref(p))
+
+
+def absa_remainder_attention(p, q, k, v, plan, o, ws, ws_bytes, stream):
+    return lib().absa_remainder_attention(ctypes.byref(p), q, k, v, ctypes.byref(plan), o, ws,
+                                          ws_bytes, stream)
 
 
 def absa_dense_reference(p, q, k, v, o, status, stream):

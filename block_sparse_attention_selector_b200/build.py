@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libabsa.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
-SOURCES = ["api.cu", "select.cu", "score.cu", "sample.cu", "attention.cu", "attention_pair.cu"]
+SOURCES = ["api.cu", "select.cu", "score.cu", "sample.cu", "attention.cu", "attention_pair.cu", "remainder.cu"]
 HEADERS = ["absa_device.cuh", "absa_kernels.cuh"]
 
 NVCC_FLAGS = [

@@ -43,12 +43,31 @@ cudaError_t launch_wait_selftest(int32_t *status, long long limit_cycles, cudaSt
 // box; tk / tv: k / v with a 64 x 4 box (sparse: one 4-token block per box)
 // or a 64 x kAttnTileKeys box (dense tiles).
 constexpr int kAttnTileKeys = 64;
+
+// Remainder mode of K5 (ESTRA-style): after the plan's tiles, tiles of 64
+// group representatives (groups of kRemGroupBlocks consecutive key blocks).
+constexpr int kRemGroupBlocks = 32;
+constexpr int kRemMaxGroups = (kSampleMaxKvBlocks + kRemGroupBlocks - 1) / kRemGroupBlocks;
+struct RemainderArgs {
+    CUtensorMap tm_mu, tm_nu;  // group mean keys / values, [B*H*G, d] bf16, 64-row boxes
+    const float *gvar;         // [B*H*G] key variance per dimension, averaged over dimensions
+    const int32_t *gcnt;       // [B*H*G] tokens per group
+    int ngroups;               // G, groups per head
+    float var_coef;            // softmax_scale^2 / 2 * log2(e)
+};
+// K7a: the group statistics of K and V for the remainder mode.
+cudaError_t launch_group_stats(const __nv_bfloat16 *k, const __nv_bfloat16 *v, int64_t BH, int N,
+                               int d, int ngroups, __nv_bfloat16 *mu, __nv_bfloat16 *nu,
+                               float *gvar, int32_t *gcnt, cudaStream_t stream);
+
+// rem != nullptr selects the remainder mode (sparse only).
 cudaError_t launch_attention(bool dense, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, const __nv_bfloat16 *k,
                              const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N, int nqb,
                              int nkb, int d, float softmax_scale, const int32_t *counts,
                              const int32_t *kv_index, const float *log_pi, int cap,
-                             int32_t *status, cudaStream_t stream);
+                             int32_t *status, cudaStream_t stream,
+                             const RemainderArgs *rem = nullptr);
 
 // K5 under the paired design: one CTA per pair of query blocks (2p, 2p+1) of
 // a head, gathering the union of the two plan rows once.  The union list is

@@ -304,7 +304,8 @@ absa_status sample_plan_run(const absa_params *p, const float *scores, const abs
 
 absa_status attention_run(const absa_params *p, const void *q, const void *k, const void *v,
                           const absa_plan *plan, void *o, int32_t *status, HeadRun hr,
-                          cudaStream_t s, bool pairs = false) {
+                          cudaStream_t s, bool pairs = false,
+                          const RemainderArgs *rem = nullptr) {
     const Dims dm = dims_of(p);
     const int64_t off = hr.bh0 * p->N * (int64_t)p->d;
     const auto *qh = static_cast<const __nv_bfloat16 *>(q) + off;
@@ -333,7 +334,32 @@ absa_status attention_run(const absa_params *p, const void *q, const void *k, co
     return from_cuda(launch_attention(false, tq, tk, tv, kh, vh, oh, hr.nbh, p->N, dm.nqb,
                                       dm.nkb, p->d, p->softmax_scale, plan->counts + row0,
                                       plan->kv_index + row0 * cap, plan->log_pi + row0 * cap,
-                                      plan->capacity, plan->status, s));
+                                      plan->capacity, plan->status, s, rem));
+}
+
+// Workspace of the remainder attention: mean keys and values (bf16) of every
+// group, then its key variance (f32) and token count (i32).
+struct RemLayout {
+    size_t mu, nu, gvar, gcnt, total;
+    int64_t ngroups;
+};
+RemLayout rem_layout(const absa_params *p) {
+    const Dims dm = dims_of(p);
+    RemLayout L;
+    L.ngroups = (dm.nkb + kRemGroupBlocks - 1) / kRemGroupBlocks;
+    const size_t n = (size_t)dm.BH * L.ngroups;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) & ~(size_t)255;
+        return o;
+    };
+    L.mu = take(n * p->d * 2);
+    L.nu = take(n * p->d * 2);
+    L.gvar = take(n * 4);
+    L.gcnt = take(n * 4);
+    L.total = off;
+    return L;
 }
 
 absa_status check_select_ws(const absa_params *p, const void *ws, size_t ws_bytes) {
@@ -516,6 +542,48 @@ absa_status absa_sparse_attention_pairs(const absa_params *p, const void *q, con
     if (2 * (int64_t)plan->capacity > kPairUnionMax) return ABSA_ERR_UNSUPPORTED;
     return attention_run(p, q, k, v, plan, o, plan->status, all_heads(p),
                          reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+size_t absa_remainder_workspace_bytes(const absa_params *p) {
+    if (absa_check_params(p) != ABSA_OK) return 0;
+    return rem_layout(p).total;
+}
+
+absa_status absa_remainder_attention(const absa_params *p, const void *q, const void *k,
+                                     const void *v, const absa_plan *plan, void *o, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    NvtxRange range("absa_remainder_attention");
+    absa_status st = absa_check_params(p);
+    if (st != ABSA_OK) return st;
+    st = check_plan(p, plan);
+    if (st != ABSA_OK) return st;
+    if (!q || !k || !v || !o || !ws) return ABSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws))
+        return ABSA_ERR_INVALID_ARG;
+    const RemLayout L = rem_layout(p);
+    if (ws_bytes < L.total) return ABSA_ERR_WORKSPACE;
+    const Dims dm = dims_of(p);
+    const auto s = reinterpret_cast<cudaStream_t>(stream);
+    auto *base = static_cast<uint8_t *>(ws);
+    auto *mu = reinterpret_cast<__nv_bfloat16 *>(base + L.mu);
+    auto *nu = reinterpret_cast<__nv_bfloat16 *>(base + L.nu);
+    auto *gvar = reinterpret_cast<float *>(base + L.gvar);
+    auto *gcnt = reinterpret_cast<int32_t *>(base + L.gcnt);
+    cudaError_t e = launch_group_stats(static_cast<const __nv_bfloat16 *>(k),
+                                       static_cast<const __nv_bfloat16 *>(v), dm.BH, p->N, p->d,
+                                       (int)L.ngroups, mu, nu, gvar, gcnt, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    RemainderArgs ra;
+    memset(&ra, 0, sizeof(ra));
+    if (!make_map_bf16(&ra.tm_mu, mu, dm.BH * L.ngroups, p->d, kAttnTileKeys) ||
+        !make_map_bf16(&ra.tm_nu, nu, dm.BH * L.ngroups, p->d, kAttnTileKeys))
+        return ABSA_ERR_CUDA;
+    ra.gvar = gvar;
+    ra.gcnt = gcnt;
+    ra.ngroups = (int)L.ngroups;
+    ra.var_coef = (float)(0.5 * (double)p->softmax_scale * (double)p->softmax_scale *
+                          1.4426950408889634);
+    return attention_run(p, q, k, v, plan, o, plan->status, all_heads(p), s, false, &ra);
 }
 
 absa_status absa_dense_reference(const absa_params *p, const void *q, const void *k,

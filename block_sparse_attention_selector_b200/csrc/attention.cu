@@ -92,14 +92,14 @@ __device__ __noinline__ void rescale_o(uint32_t o_t, float alpha) {
 // The logit bias of tile t is written together with K_t into slot t % 4 of
 // its own ring (every K loader warp arrives on b_full after writing its
 // columns), so the softmax of a tile never waits for that tile's V.
-template <int D, bool DENSE>
+template <int D, bool DENSE, bool REM>
 __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ k,
     const __nv_bfloat16 *__restrict__ v, __nv_bfloat16 *__restrict__ o, int N, int nqb,
     int nkb, float scale_log2, const int32_t *__restrict__ counts,
     const int32_t *__restrict__ kv_index, const float *__restrict__ log_pi, int cap,
-    int32_t *status) {
+    int32_t *status, const __grid_constant__ RemainderArgs rem) {
     using S = AttnSmem<D>;
     extern __shared__ uint8_t attn_smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -118,6 +118,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
     int *bad_flag = reinterpret_cast<int *>(bars + 21);  // a plan entry out of range
+    // remainder mode: per tile slot the representatives' variance terms
+    // (64 floats after the bias ring) and the plan's tokens per group
+    float *cvar_s = reinterpret_cast<float *>(sm + S::kBytes);
+    int *gsel = reinterpret_cast<int *>(sm + S::kBytes + kBiasStages * kTileKeys * 4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             mbar_init(pv_done + s, 1);
         }
         for (int i = 0; i < kBiasStages; ++i) mbar_init(b_full + i, DENSE ? 1 : kKLoadWarps);
+        static_assert(!(DENSE && REM), "the remainder mode extends the sparse mode");
         *abort_flag = 0;
         *bad_flag = 0;
         mbar_fence_init();
@@ -158,7 +163,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             count = 0;
         }
     }
-    const int T = (count + kTileBlocks - 1) / kTileBlocks;
+    const int Ts = (count + kTileBlocks - 1) / kTileBlocks;  // tiles of plan blocks
+    // remainder mode: then one tile per 64 group representatives
+    const int T = Ts + (REM ? (rem.ngroups + kTileKeys - 1) / kTileKeys : 0);
+    if (REM) {  // tokens of the plan's blocks per group
+        for (int g = tid; g < rem.ngroups; g += kAttnThreads) gsel[g] = 0;
+        __syncthreads();
+        const int32_t *ir = kv_index + row * cap;
+        for (int e = tid; e < count; e += kAttnThreads) {
+            const int b = __ldg(ir + e);
+            if (b >= 0 && b < nkb) atomicAdd(&gsel[b / kRemGroupBlocks], min(4, N - 4 * b));
+        }
+    }
     // Rows of a partial tile that no box overwrites must hold finite values
     // (P = 0 there, and 0 * NaN would poison O).  After its first use a ring
     // stage holds finite stale rows, so only a row whose first two tiles are
@@ -226,7 +242,36 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                 return false;
             float *bias = bias_s + (t % kBiasStages) * kTileKeys;
             const uint32_t k_s = smem_u32(sm + S::kKOff + st * S::kKVBytes);
-            if (DENSE) {
+            if (REM && t >= Ts) {
+                // a tile of 64 group representatives: mean keys, log2 of the
+                // tokens left outside the plan, and the variance term
+                const int g0 = kTileKeys * (t - Ts);
+                const int64_t gb = bh * rem.ngroups;
+                if (lw == 0) {
+                    float bb[2], cc[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int g = g0 + 2 * lane + h;
+                        const bool in = g < rem.ngroups;
+                        const int left = in ? __ldg(rem.gcnt + gb + g) - gsel[g] : 0;
+                        bb[h] = left > 0 ? log2f((float)left) : -INFINITY;
+                        cc[h] = in ? rem.var_coef * __ldg(rem.gvar + gb + g) : 0.f;
+                    }
+                    reinterpret_cast<float2 *>(bias)[lane] = make_float2(bb[0], bb[1]);
+                    reinterpret_cast<float2 *>(cvar_s + (t % kBiasStages) * kTileKeys)[lane] =
+                        make_float2(cc[0], cc[1]);
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(b_full + t % kBiasStages);
+                    if (lw == 0) {
+                        mbar_arrive_expect_tx(k_full + st, S::kKVBytes);
+                        for (int r = 0; r < R; ++r)
+                            tma_load_2d(k_s + r * S::kKVRegion, &rem.tm_mu, 64 * r,
+                                        (int)(gb + g0), k_full + st);
+                    }
+                }
+            } else if (DENSE) {
                 if (lw == 0) {
                     float2 bb;
                     const int t0 = kTileKeys * t + 2 * lane;
@@ -246,7 +291,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                 if (has_box && reg == 0) {  // logit bias of the block's 4 columns
                     float4 bb = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
                     if (b >= 0) {
-                        const float sh = -lpv * kLog2e;
+                        const float sh = REM ? 0.f : -lpv * kLog2e;  // remainder mode: no HT shift
                         const int t0 = 4 * b;
                         bb.x = t0 < N ? sh : -INFINITY;
                         bb.y = t0 + 1 < N ? sh : -INFINITY;
@@ -275,7 +320,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                                                              status, abort_flag, kLoaderPolls)))
                 return false;
             const uint32_t v_s = smem_u32(sm + S::kVOff + st * S::kKVBytes);
-            if (DENSE) {
+            if (REM && t >= Ts) {  // the representatives' mean values
+                if (gw == 0 && lane == 0) {
+                    mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
+                    for (int r = 0; r < R; ++r)
+                        tma_load_2d(v_s + r * S::kKVRegion, &rem.tm_nu, 64 * r,
+                                    (int)(bh * rem.ngroups + kTileKeys * (t - Ts)), v_full + st);
+                }
+            } else if (DENSE) {
                 if (gw == 0 && lane == 0) {
                     mbar_arrive_expect_tx(v_full + st, S::kKVBytes);
                     for (int r = 0; r < R; ++r)
@@ -349,7 +401,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             };
             bool ok = mbar_wait(q_full, 0, status, abort_flag) && issue_s(0);
             if (ok && T > 1) ok = issue_s(1);
-            for (int j = 0; j < T && ok; ++j) {
+            for (int j = 0; j < T; ++j) {
                 ok = issue_pv(j);
                 if (ok && j + 2 < T)
                     ok = mbar_wait(pv_done + (j & 1), (j >> 1) & 1, status, abort_flag) &&
@@ -367,6 +419,28 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
         const uint32_t o_t = tmem_o + lane_base;
         float m_ref = -INFINITY, lsum = 0.f;
         bool ok = true;
+        // remainder mode: |q_r|^2 for the representatives' variance term, from
+        // this row of the Q tile (the swizzle only permutes the row's 16-byte
+        // chunks; lane r starts at chunk r so that the lanes spread over banks)
+        uint64_t qn2 = 0;
+        if (REM && T > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, status, abort_flag));
+            float qn = 0.f;
+#pragma unroll 1
+            for (int rr = 0; rr < S::kRegions; ++rr)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(
+                        sm + S::kQOff + rr * S::kQRegion + r * 128 + ((c + r) & 7) * 16);
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xFFFF0000u);
+                        qn = fmaf(lo, lo, fmaf(hi, hi, qn));
+                    }
+                }
+            qn2 = ((uint64_t)__float_as_uint(qn) << 32) | __float_as_uint(qn);
+        }
         for (int j = 0; j < T; ++j) {
             const int b = j & 1;
             const uint32_t s_t = tmem + lane_base + b * kTileKeys;
@@ -382,6 +456,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                             mbar_wait(b_full + bs, (j / kBiasStages) & 1, status, abort_flag));
             if (!ok) break;
             const uint32_t bias_u = smem_u32(bias_s + bs * kTileKeys);
+            const uint32_t cvar_u = REM ? smem_u32(cvar_s + bs * kTileKeys) : 0u;
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             const uint64_t sc2 =
                 ((uint64_t)__float_as_uint(scale_log2) << 32) | __float_as_uint(scale_log2);
@@ -393,6 +468,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                     asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
                                  : "=l"(b01), "=l"(b23)
                                  : "r"(bias_u + (uint32_t)(ch * 32 + i) * 4u));
+                    if (REM && j >= Ts) {  // + |q|^2 times the variance term
+                        uint64_t c01, c23;
+                        asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
+                                     : "=l"(c01), "=l"(c23)
+                                     : "r"(cvar_u + (uint32_t)(ch * 32 + i) * 4u));
+                        b01 = f32x2_fma(c01, qn2, b01);
+                        b23 = f32x2_fma(c23, qn2, b23);
+                    }
                     const uint64_t x01 =
                         f32x2_fma(((uint64_t)sv[ch][i + 1] << 32) | sv[ch][i], sc2, b01);
                     const uint64_t x23 =
@@ -501,24 +584,26 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
     }
 }
 
-template <int D, bool DENSE>
+template <int D, bool DENSE, bool REM>
 static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &tk,
                                       const CUtensorMap &tv, const __nv_bfloat16 *k,
                                       const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N,
                                       int nqb, int nkb, float scale_log2, const int32_t *counts,
                                       const int32_t *kv_index, const float *log_pi, int cap,
-                                      int32_t *status, cudaStream_t stream) {
-    const int smem = AttnSmem<D>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE>,
+                                      int32_t *status, const RemainderArgs &rem,
+                                      cudaStream_t stream) {
+    // remainder mode: the variance-term ring and the per-group plan tokens follow
+    const int smem = AttnSmem<D>::kAlloc + (REM ? kBiasStages * kTileKeys * 4 + kRemMaxGroups * 4 : 0);
+    cudaError_t e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE, REM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     // two CTAs per SM: ask for the largest shared-memory carveout
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE>,
+        e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE, REM>,
                                  cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    absa_attention_kernel<D, DENSE><<<(unsigned)(BH * nqb), kAttnThreads, smem, stream>>>(
-        tq, tk, tv, k, v, o, N, nqb, nkb, scale_log2, counts, kv_index, log_pi, cap, status);
+    absa_attention_kernel<D, DENSE, REM><<<(unsigned)(BH * nqb), kAttnThreads, smem, stream>>>(
+        tq, tk, tv, k, v, o, N, nqb, nkb, scale_log2, counts, kv_index, log_pi, cap, status, rem);
     return cudaGetLastError();
 }
 
@@ -527,17 +612,23 @@ cudaError_t launch_attention(bool dense, const CUtensorMap &tq, const CUtensorMa
                              const __nv_bfloat16 *v, __nv_bfloat16 *o, int64_t BH, int N, int nqb,
                              int nkb, int d, float softmax_scale, const int32_t *counts,
                              const int32_t *kv_index, const float *log_pi, int cap,
-                             int32_t *status, cudaStream_t stream) {
+                             int32_t *status, cudaStream_t stream, const RemainderArgs *rem) {
     const float sl2 = softmax_scale * kLog2e;
-    if (d == 64)
-        return dense ? launch_attention_d<64, true>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
-                                                    kv_index, log_pi, cap, status, stream)
-                     : launch_attention_d<64, false>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
-                                                     kv_index, log_pi, cap, status, stream);
-    return dense ? launch_attention_d<128, true>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
-                                                 kv_index, log_pi, cap, status, stream)
-                 : launch_attention_d<128, false>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,
-                                                  kv_index, log_pi, cap, status, stream);
+    RemainderArgs none;
+    memset(&none, 0, sizeof(none));
+    const RemainderArgs &ra = rem ? *rem : none;
+#define ABSA_LAUNCH(DD, DN, RM)                                                                    \
+    return launch_attention_d<DD, DN, RM>(tq, tk, tv, k, v, o, BH, N, nqb, nkb, sl2, counts,      \
+                                          kv_index, log_pi, cap, status, ra, stream)
+    if (d == 64) {
+        if (dense) ABSA_LAUNCH(64, true, false);
+        if (rem) ABSA_LAUNCH(64, false, true);
+        ABSA_LAUNCH(64, false, false);
+    }
+    if (dense) ABSA_LAUNCH(128, true, false);
+    if (rem) ABSA_LAUNCH(128, false, true);
+    ABSA_LAUNCH(128, false, false);
+#undef ABSA_LAUNCH
 }
 
 }  // namespace absa

@@ -238,6 +238,38 @@ absa_status absa_sparse_attention_pairs(const absa_params *p, const void *q, con
                                         const void *v, const absa_plan *plan, void *o,
                                         void *stream);
 
+/* Bytes of workspace absa_remainder_attention needs (0 if p is invalid).
+ * With G = ceil(NKB / 32) groups per head, each region at a 256-byte
+ * boundary in this order:
+ *   mu    bf16 [B,H,G,d]  mean key of each group's tokens
+ *   nu    bf16 [B,H,G,d]  mean value
+ *   var   f32  [B,H,G]    key variance per dimension, averaged over d
+ *   count i32  [B,H,G]    tokens in the group (128, fewer in a head's last) */
+size_t absa_remainder_workspace_bytes(const absa_params *p);
+
+/* ESTRA-style attention (ESTRA page, summary and figure: the selected pairs
+ * exact, the rest from group averages with a variance-calibrated correction
+ * of the representatives' weights), on the plan of this library.  For every
+ * valid query i of block qb, one softmax runs over
+ *   - the tokens t of the plan row's blocks, logit s q_i.k_t (no ln pi shift:
+ *     the plan's blocks are the exact part), and
+ *   - one representative per group g of 32 consecutive key blocks (128
+ *     tokens), key mu_g and value nu_g (the group's mean key and value),
+ *     logit s q_i.mu_g + s^2 |q_i|^2 var_g / 2 + ln(m_g), where m_g is the
+ *     number of the group's tokens outside the plan row (no representative if
+ *     m_g = 0) and var_g the group's key variance per dimension averaged over
+ *     dimensions (the Gaussian moment identity E exp(X) = exp(E X + Var X / 2)
+ *     with an isotropic key spread),
+ * with s = softmax_scale.  The group statistics are written to ws first
+ * (ws_bytes >= absa_remainder_workspace_bytes(p), ABSA_ERR_WORKSPACE
+ * otherwise), then the attention kernel runs the plan's tiles followed by
+ * ceil(G / 64) tiles of representatives in the same softmax.  Plan checks,
+ * bad rows and status as absa_sparse_attention; repeated plan entries are
+ * counted as often as they appear. */
+absa_status absa_remainder_attention(const absa_params *p, const void *q, const void *k,
+                                     const void *v, const absa_plan *plan, void *o, void *ws,
+                                     size_t ws_bytes, void *stream);
+
 /* Dense softmax attention (the full-attention reference of the pages'
  * evaluation) with the same tile machinery over contiguous keys.  status is
  * a device word for ABSA_DEVFLAG_TIMEOUT (may be NULL). */

@@ -113,6 +113,14 @@ def test_entry_points_reject_null_and_misaligned_pointers_before_cuda(L):
                  None) == _abi.ABSA_ERR_INVALID_ARG
     wide = _abi.absa_plan(4, 128, 3073, 16, 16, 16, 16, 16)
     assert pairs(p, 16, 16, 16, wide, 16, None) == _abi.ABSA_ERR_UNSUPPORTED
+    # the remainder attention: workspace size, null and short workspaces
+    rb = _abi.absa_remainder_workspace_bytes(p)
+    assert rb > 0 and _abi.absa_remainder_workspace_bytes(_p(N=0)) == 0
+    rem = _abi.absa_remainder_attention
+    ok_plan = _abi.absa_plan(4, 128, 96, 16, 16, 16, 16, 16)
+    assert rem(p, 16, 16, 16, ok_plan, 16, None, rb, None) == _abi.ABSA_ERR_INVALID_ARG
+    assert rem(p, 16, 16, 16, ok_plan, 16, 16, rb - 1, None) == _abi.ABSA_ERR_WORKSPACE
+    assert rem(p, 16, 16, 16, bad, 16, 16, rb, None) == _abi.ABSA_ERR_INVALID_ARG
     # the host-buffer step: null host pointers, an empty head run, a short workspace
     good = _abi.absa_plan(4, 128, 96, 16, 16, 16, 16, 16)
     step = _abi.absa_step_host
