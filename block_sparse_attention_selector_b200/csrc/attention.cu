@@ -170,9 +170,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
         for (int g = tid; g < rem.ngroups; g += kAttnThreads) gsel[g] = 0;
         __syncthreads();
         const int32_t *ir = kv_index + row * cap;
-        for (int e = tid; e < count; e += kAttnThreads) {
-            const int b = __ldg(ir + e);
-            if (b >= 0 && b < nkb) atomicAdd(&gsel[b / kRemGroupBlocks], min(4, N - 4 * b));
+        for (int e0 = tid; e0 < count; e0 += 4 * kAttnThreads) {  // 4 entry loads in flight
+            int bq[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                bq[u] = e0 + u * kAttnThreads < count ? __ldg(ir + e0 + u * kAttnThreads) : -1;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (bq[u] >= 0 && bq[u] < nkb)
+                    atomicAdd(&gsel[bq[u] / kRemGroupBlocks], min(4, N - 4 * bq[u]));
         }
     }
     // Rows of a partial tile that no box overwrites must hold finite values
@@ -422,7 +428,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
         // remainder mode: |q_r|^2 for the representatives' variance term, from
         // this row of the Q tile (the swizzle only permutes the row's 16-byte
         // chunks; lane r starts at chunk r so that the lanes spread over banks)
-        uint64_t qn2 = 0;
+        float *qn_s = reinterpret_cast<float *>(gsel + kRemMaxGroups);  // [128] |q_r|^2
         if (REM && T > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, status, abort_flag));
             float qn = 0.f;
@@ -439,7 +445,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                         qn = fmaf(lo, lo, fmaf(hi, hi, qn));
                     }
                 }
-            qn2 = ((uint64_t)__float_as_uint(qn) << 32) | __float_as_uint(qn);
+            // read back per group tile, divided by the logit scale (no term at scale 0)
+            qn_s[r] = scale_log2 != 0.f ? qn / scale_log2 : 0.f;
         }
         for (int j = 0; j < T; ++j) {
             const int b = j & 1;
@@ -457,6 +464,27 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
             if (!ok) break;
             const uint32_t bias_u = smem_u32(bias_s + bs * kTileKeys);
             const uint32_t cvar_u = REM ? smem_u32(cvar_s + bs * kTileKeys) : 0u;
+            if (REM && j >= Ts) {
+                // representatives: fold |q_r|^2 c_g into S (S += |q_r|^2 c_g / scale),
+                // so that the loop below stays the one of the plan's tiles
+                const float qs = qn_s[r];
+                const uint64_t qs2 = ((uint64_t)__float_as_uint(qs) << 32) | __float_as_uint(qs);
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        uint64_t c01, c23;
+                        asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
+                                     : "=l"(c01), "=l"(c23)
+                                     : "r"(cvar_u + (uint32_t)(ch * 32 + i) * 4u));
+                        const uint64_t s01 = f32x2_fma(c01, qs2, ((uint64_t)sv[ch][i + 1] << 32) | sv[ch][i]);
+                        const uint64_t s23 = f32x2_fma(c23, qs2, ((uint64_t)sv[ch][i + 3] << 32) | sv[ch][i + 2]);
+                        sv[ch][i] = (uint32_t)s01;
+                        sv[ch][i + 1] = (uint32_t)(s01 >> 32);
+                        sv[ch][i + 2] = (uint32_t)s23;
+                        sv[ch][i + 3] = (uint32_t)(s23 >> 32);
+                    }
+            }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             const uint64_t sc2 =
                 ((uint64_t)__float_as_uint(scale_log2) << 32) | __float_as_uint(scale_log2);
@@ -468,14 +496,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
                     asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
                                  : "=l"(b01), "=l"(b23)
                                  : "r"(bias_u + (uint32_t)(ch * 32 + i) * 4u));
-                    if (REM && j >= Ts) {  // + |q|^2 times the variance term
-                        uint64_t c01, c23;
-                        asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
-                                     : "=l"(c01), "=l"(c23)
-                                     : "r"(cvar_u + (uint32_t)(ch * 32 + i) * 4u));
-                        b01 = f32x2_fma(c01, qn2, b01);
-                        b23 = f32x2_fma(c23, qn2, b23);
-                    }
                     const uint64_t x01 =
                         f32x2_fma(((uint64_t)sv[ch][i + 1] << 32) | sv[ch][i], sc2, b01);
                     const uint64_t x23 =
@@ -593,7 +613,8 @@ static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &
                                       int32_t *status, const RemainderArgs &rem,
                                       cudaStream_t stream) {
     // remainder mode: the variance-term ring and the per-group plan tokens follow
-    const int smem = AttnSmem<D>::kAlloc + (REM ? kBiasStages * kTileKeys * 4 + kRemMaxGroups * 4 : 0);
+    const int smem =
+        AttnSmem<D>::kAlloc + (REM ? kBiasStages * kTileKeys * 4 + kRemMaxGroups * 4 + 128 * 4 : 0);
     cudaError_t e = cudaFuncSetAttribute(absa_attention_kernel<D, DENSE, REM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     // two CTAs per SM: ask for the largest shared-memory carveout
