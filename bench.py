@@ -56,6 +56,10 @@ def parse():
     ap.add_argument("--sampling", default="poisson", choices=["poisson", "systematic", "paired"],
                     help="SIP design: Poisson draws (default), systematic (exactly n blocks) or "
                          "paired (Poisson draws shared by query blocks 2p and 2p+1)")
+    ap.add_argument("--remainder", action="store_true",
+                    help="also time absa_remainder_attention (ESTRA-style remainder) on the "
+                         "step's plan and report both estimators' relative L2 to dense attention")
+    ap.add_argument("--remainder-steps", type=int, default=5)
     ap.add_argument("--harness", action="store_true",
                     help="mass-retention / error harness on the 480p and 720p layers (JSON lines; "
                          "no main line)")
@@ -420,6 +424,31 @@ def run_ours(args):
         torch.cuda.synchronize()
         dense_ms.append(ev_d[0].elapsed_time(ev_d[1]))
 
+    # ESTRA-style remainder attention on the step's plan (group statistics and
+    # the attention's remainder mode), and both estimators against dense attention
+    rem = None
+    if args.remainder:
+        rws = torch.empty(absa.absa_remainder_workspace_bytes(p), dtype=torch.uint8, device=dev)
+        o_r = torch.empty_like(o)
+        ev_r = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        rem_ms = []
+        for i in range(3 + args.remainder_steps):
+            flush.zero_()
+            ev_r[0].record(stream)
+            absa.remainder_attention(p, q, k, v, plan, o_r, ws=rws, stream=stream)
+            ev_r[1].record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                rem_ms.append(ev_r[0].elapsed_time(ev_r[1]))
+        o_d = absa.dense_reference(p, q, k, v, stream=stream)
+        o_s = absa.sparse_attention(p, q, k, v, plan, stream=stream)
+        torch.cuda.synchronize()
+        nd = float(torch.linalg.vector_norm(o_d.float()))
+        rem = {"ms": float(np.median(rem_ms)), "launches": 2,
+               "rel_l2_vs_dense": float(torch.linalg.vector_norm(o_r.float() - o_d.float())) / nd,
+               "ht_rel_l2_vs_dense": float(torch.linalg.vector_norm(o_s.float() - o_d.float())) / nd}
+        del o_r, o_d, o_s, rws
+
     # end to end through the public API with host buffers: absa_step_host copies
     # runs of heads in on one stream, computes them on `stream` and copies their
     # outputs back on a third, so the transfers overlap the kernels
@@ -475,6 +504,7 @@ def run_ours(args):
                 "dense_tflops": (4.0 * w.d * w.N * w.N * w.B * w.H / (np.median(dense_ms) * 1e-3)
                                  / 1e12) if dense_ms else None,
                 "mean_blocks_per_row": float(counts.mean()),
+                "remainder_attention": rem,
             },
             "roofline": {"bound": "tensor", "kernel": "absa_attention_kernel<128,sparse>",
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
