@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
     // which read them anyway: such an entry loads block 0 instead and the row
     // is written as zeros at the end.
     int count;
+    bool count_bad = false;
     if (DENSE) {
         count = nkb;
     } else {
@@ -161,11 +162,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2) absa_attention_kernel(
         if (count < 0 || count > cap) {
             if (tid == 0) atomicOr(status, ABSA_DEVFLAG_BAD_PLAN);
             count = 0;
+            count_bad = true;
         }
     }
     const int Ts = (count + kTileBlocks - 1) / kTileBlocks;  // tiles of plan blocks
-    // remainder mode: then one tile per 64 group representatives
-    const int T = Ts + (REM ? (rem.ngroups + kTileKeys - 1) / kTileKeys : 0);
+    // remainder mode: then one tile per 64 group representatives (none for a
+    // rejected row, which is written as zeros)
+    const int T = Ts + (REM && !count_bad ? (rem.ngroups + kTileKeys - 1) / kTileKeys : 0);
     if (REM) {  // tokens of the plan's blocks per group
         for (int g = tid; g < rem.ngroups; g += kAttnThreads) gsel[g] = 0;
         __syncthreads();

@@ -82,13 +82,14 @@ def test_remainder_bad_rows_and_short_workspace():
     ref = oracle.sample_plan(s_ref, w.budget, 1, oracle.plan_capacity(w.budget, w.nkb))
     plan = plan_from_oracle(p, ref)
     plan.kv_index[0, 1, 2, 0] = w.nkb  # an index out of range: that row is zeroed
+    plan.counts[0, 0, 3] = plan.capacity + 1  # a count above capacity: zeroed as well
     qd, kd, vd = device_bf16(q), device_bf16(k), device_bf16(v)
     o = remainder_attention(p, qd, kd, vd, plan)
     with pytest.raises(AbsaError) as e:
         plan.check()
     assert e.value.code == _abi.ABSA_ERR_BAD_PLAN
     o = o.float().cpu().numpy()
-    assert np.all(o[0, 1, 256:384] == 0)
+    assert np.all(o[0, 1, 256:384] == 0) and np.all(o[0, 0, 384:512] == 0)
     short = torch.empty(_abi.absa_remainder_workspace_bytes(p) - 256, dtype=torch.uint8,
                         device="cuda")
     with pytest.raises(AbsaError) as e:
