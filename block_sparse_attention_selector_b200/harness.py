@@ -24,7 +24,8 @@ attention and score computation runs in the library's kernels.
 """
 import math
 
-from . import Plan, dense_reference, params_for, sample_plan, select_scores, sparse_attention
+from . import (Plan, dense_reference, params_for, remainder_attention, sample_plan, select_scores,
+               sparse_attention)
 
 
 def block_masses(p, q, k, chunk_out=None):
@@ -151,6 +152,10 @@ def retention_report(w, q, k, v, budget=None, seed=0):
     det("block_mean", _topn(block_mean_scores(p, q, k), n))
     scores, _ = select_scores(p, q, k)
     det("ibcs_topn", _topn(scores, n))
+    # ESTRA-style remainder (the plan's blocks exact, the rest through group
+    # representatives) on the IBCS top-n selection
+    out["rel_l2_remainder_ibcs_topn"] = rel_l2(
+        remainder_attention(p, q, k, v, plan_from_indices(p, _topn(scores, n))), o_dense)
 
     # 128-token key blocks at the same key fraction
     n128 = max(1, round(n / 32))
@@ -170,6 +175,9 @@ def retention_report(w, q, k, v, budget=None, seed=0):
             out[f"pair_union_over_own_{design}"] = pair_union_ratio(plan, nkb)
         o = sparse_attention(ps, q, k, v, plan)
         out[f"rel_l2_sip_{design}"] = rel_l2(o, o_dense)
+        if design == "poisson":  # the remainder estimator on the same sampled blocks
+            out["rel_l2_remainder_sip_poisson"] = rel_l2(remainder_attention(ps, q, k, v, plan),
+                                                         o_dense)
 
     top = out["mass_ideal_topk"]
     out["recall_gap_block_mean"] = top - out["mass_block_mean"]

@@ -71,6 +71,6 @@ def test_retention_report_invariants(w):
                 "mass_sip_systematic", "mass_sip_paired"):
         assert abs(full[key] - 1.0) < 1e-2, (key, full[key])
     for key in ("rel_l2_ideal_topk", "rel_l2_sip_poisson", "rel_l2_sip_systematic",
-                "rel_l2_sip_paired"):
+                "rel_l2_sip_paired", "rel_l2_remainder_ibcs_topn", "rel_l2_remainder_sip_poisson"):
         assert full[key] == 0.0, (key, full[key])
     assert full["pair_union_over_own_paired"] == 1.0
