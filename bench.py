@@ -67,7 +67,9 @@ def parse():
                     help="heads of the 720p layers in the harness (the 480p layer uses --heads or "
                          "all 40)")
     ap.add_argument("--sweep", action="store_true",
-                    help="density sweep and 16-step plan-reuse schedule (JSON lines; no main line)")
+                    help="density sweep (1, 2, 5, 10, 25, 100%% of the layer's key blocks) and the "
+                         "16-step plan-reuse schedule (JSON lines; no main line); the sweep "
+                         "configuration is --workload wan480")
     return ap.parse_args()
 
 
@@ -536,7 +538,12 @@ def run_ours(args):
 
 # ------------------------------------------------------------------ sweep
 
-SWEEP_BUDGETS = (82, 164, 410, 819, 2048, 8190)  # round-half-up of 1, 2, 5, 10, 25, 100% of 8190
+def sweep_budgets(w):
+    """Budgets of the density sweep: round-half-up of 1, 2, 5, 10, 25 and 100% of the layer's
+    key blocks (82 ... 8190 on the Wan2.1 480p layer, the sweep configuration)."""
+    from block_sparse_attention_selector_b200 import synthetic
+
+    return tuple(int(math.floor(f * w.nkb + 0.5)) for f in synthetic.SWEEP_FRACTIONS)
 
 
 def run_sweep(args):
@@ -580,7 +587,7 @@ def run_sweep(args):
         o_dense, dense_ms = timed(lambda: absa.dense_reference(p0, q, k, v))
     dense_rms = float(o_dense.float().pow(2).mean().sqrt())
     v_rms = float(v.float().pow(2).mean().sqrt())
-    for budget, design in [(b, d) for b in SWEEP_BUDGETS for d in ("poisson", "systematic")]:
+    for budget, design in [(b, d) for b in sweep_budgets(w) for d in ("poisson", "systematic")]:
         sel, att, rel, err, blocks = [], [], [], [], []
         for seed in range(8):
             p = absa.params_for(w, seed=seed, budget=budget, sampling=design)
