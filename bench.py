@@ -653,8 +653,10 @@ def run_harness(args):
     from block_sparse_attention_selector_b200 import harness, synthetic
 
     dev = torch.device("cuda", 0)
-    layers = [workload(args.heads)]
+    layers = [workload(args.heads, args.workload)]
     for w in (synthetic.WAN720, synthetic.HUNYUAN720):
+        if w.name == layers[0].name:
+            continue
         h = min(w.H, args.harness_heads)
         layers.append(dataclasses.replace(w, H=h, name=f"{w.name}_{h}heads") if h < w.H else w)
     for w in layers:
