@@ -66,6 +66,17 @@ def test_workspace_bytes_covers_layout(L):
     assert need <= got <= need + 11 * 256
 
 
+@pytest.mark.parametrize("w", [synthetic.TOY, synthetic.WAN480, synthetic.HUNYUAN720],
+                         ids=lambda w: w.name)
+def test_remainder_workspace_bytes_match_the_documented_layout(L, w):
+    """mu, nu (bf16 [B,H,G,d]), var and count ([B,H,G], 4 bytes each), every region at a
+    256-byte boundary, G = ceil(NKB / 32)."""
+    G = (w.nkb + 31) // 32
+    n = w.B * w.H * G
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert _abi.absa_remainder_workspace_bytes(_p(w)) == 2 * up(n * w.d * 2) + 2 * up(n * 4)
+
+
 @pytest.mark.parametrize("field,value,code", [
     ("d", 96, _abi.ABSA_ERR_UNSUPPORTED),
     ("q_block", 64, _abi.ABSA_ERR_UNSUPPORTED),
