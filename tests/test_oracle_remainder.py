@@ -119,3 +119,21 @@ def test_weight_counts_the_tokens_left():
                    np.arange(G, 2 * G, dtype=np.int32)):
         o = oracle.remainder_attention_rows(q, k, v, blocks, scale)
         np.testing.assert_allclose(o, 0.5, atol=1e-12)
+
+
+def test_repeated_entries_count_as_often_as_listed():
+    """The same two constant groups (values 0 and 1, equal keys): a block of
+    group 0 listed twice enters the exact part twice (8 tokens) and leaves the
+    rest twice (120 tokens left), so group 0 still weighs 128 against 128 and
+    the output stays 0.5; listing it 40 times empties the rest (no
+    representative) and group 0 weighs 160: the output is 128 / 288."""
+    d = 8
+    N = 8 * G
+    k = bits(np.ones((N, d)) * 0.25)
+    v = bits(np.where(np.arange(N)[:, None] < 4 * G, 0.0, 1.0) * np.ones((1, d)))
+    q = bits(np.ones((2, d)))
+    s = 1.0 / math.sqrt(d)
+    o = oracle.remainder_attention_rows(q, k, v, np.array([3, 3], np.int32), s)
+    np.testing.assert_allclose(o, 0.5, atol=1e-12)
+    o = oracle.remainder_attention_rows(q, k, v, np.full(40, 3, np.int32), s)
+    np.testing.assert_allclose(o, 128.0 / 288.0, atol=1e-12)
