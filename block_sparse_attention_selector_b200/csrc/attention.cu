@@ -26,6 +26,13 @@
 // the final O is divided by the fp32 sum of the bf16-rounded P, the weights
 // the PV product used (a row dominated by a few tokens then returns their
 // values without the rounding of P showing).
+//
+// Remainder mode (ESTRA page, summary and figure: the selected pairs exact,
+// the rest from group averages with a variance-calibrated correction): the
+// plan's tiles run with a zero bias, then tiles of 64 group representatives
+// (mean keys and values of 32-block groups, loaded as 64-row boxes) follow in
+// the same softmax chain, each with the bias log2 of its tokens outside the
+// plan row and the term |q|^2 * s^2 var / 2 added to its logits.
 #include "absa_kernels.cuh"
 
 namespace absa {
